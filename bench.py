@@ -1,0 +1,393 @@
+#!/usr/bin/env python
+"""Benchmark of the Star Attention hot path on NVIDIA B200.
+
+One step = the whole hot path over one batch of the workload, through the C ABI:
+RoPE + KV append and Phase-1 anchor-augmented attention (star_phase1_encode),
+query append + per-block partials (star_phase2_partial), the exact merge
+(star_lse_merge), and S decode steps (star_decode_step).  Inputs are seeded
+synthetic tensors already resident in HBM when the timed region starts; the
+`e2e` leg repeats the step from pinned host buffers with the copies inside the
+timed region.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl star|reference]
+
+Multi-GPU (torchrun): every rank runs its own independent sequence batch (the
+path partitions by sequence; no collective on the data path); time is the max
+over ranks.  `--impl reference` times the CPU oracle (float64 numpy) on a
+bounded sample of the same workload on the host cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import get_config, make_inputs  # noqa: E402
+
+METRIC = "Phase-1 ctx tok/s (% BF16 peak) at 128K; Phase-2 decode µs/step (HBM GB/s)"
+UNIT = "ctx tok/s"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default="llama8b-128k-b32768")
+    ap.add_argument("--impl", default="star", choices=["star", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=8, help="Phase-1 rows per block in the oracle sample")
+    return ap.parse_args()
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        return {"hbm_gbs": pk["hbm_gbs"], "bf16": pk["bf16_tflops"], "bf16_sustained": pk["bf16_tflops_sustained"],
+                "kind": "of measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "kind": "of fallback"}
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.lines = []
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            target = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            target = str(device_index)
+        self.cmd = ["nvidia-smi", "-i", target, "--query-gpu=" + ",".join(self.FIELDS),
+                    "--format=csv,noheader,nounits", "-lms", "200"]
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, smax, reasons = [], [], set()
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# The CUDA path
+# ---------------------------------------------------------------------------
+class StarRun:
+    """Buffers and the step sequence of one workload on one GPU."""
+
+    def __init__(self, wl, device):
+        import block_sparse_attention_star_b200 as star
+        self.star, self.wl, self.dev = star, wl, device
+        self.inp = make_inputs(wl, device)
+        self.shape = star.StarShape.make(B=wl.B, Hq=wl.Hq, Hkv=wl.Hkv, d=wl.d, L=wl.L, b=wl.b, T_max=wl.T_max,
+                                         page_tokens=wl.page_tokens, rope_theta=wl.theta)
+        self.cache = star.PagedKVCache(self.shape, device=device)
+        self.o_ctx = torch.empty_like(self.inp["q_ctx"])
+        self.o_part, self.lse_part = star.alloc_partials(self.shape, wl.T, device)
+        self.ws2 = star.workspace(self.shape, star.STAR_OP_PHASE2, wl.T, device)
+        self.wsd = star.workspace(self.shape, star.STAR_OP_DECODE, 0, device)
+        self.o_q = torch.empty((wl.B, wl.T, wl.Hq, wl.d), dtype=torch.bfloat16, device=device)
+        self.lse_q = torch.empty((wl.B, wl.T, wl.Hq), dtype=torch.float32, device=device)
+        self.o_dec = torch.empty((wl.S, wl.B, 1, wl.Hq, wl.d), dtype=torch.bfloat16, device=device)
+        self.lse_dec = torch.empty((wl.S, wl.B, wl.Hq), dtype=torch.float32, device=device)
+        cpb_ws = star.star_workspace_size(self.shape, star.STAR_OP_PHASE2, wl.T)
+        self.launches_per_step = 3 + 2 + (1 if cpb_ws > 0 else 0) + 1 + 3 * wl.S
+
+    def step(self, ev=None):
+        """One pass of the hot path.  ev: optional dict of (start, stop) event lists to record."""
+        s, wl, inp = self.star, self.wl, self.inp
+        if ev:
+            s.star_set_trace_events(*ev["p1"])
+        s.star_phase1_encode(self.shape, self.cache, inp["q_ctx"], inp["k_ctx"], inp["v_ctx"], inp["pos_ctx"], self.o_ctx)
+        if ev:
+            s.star_set_trace_events(*ev["p2"])
+        s.star_phase2_partial(self.shape, self.cache, inp["q_query"], inp["k_query"], inp["v_query"], inp["pos_query"],
+                              wl.T, self.o_part, self.lse_part, self.ws2)
+        if ev:
+            s.star_set_trace_events(None, None)
+        s.star_lse_merge(self.shape.n, wl.B * wl.T * wl.Hq, wl.d, self.o_part, self.lse_part, self.o_q, self.lse_q)
+        for st in range(wl.S):
+            if ev:
+                s.star_set_trace_events(*ev["dec"][st])
+                ev["dec_call"][st][0].record()
+            s.star_decode_step(self.shape, self.cache, inp["q_dec"][st], inp["k_dec"][st], inp["v_dec"][st],
+                               inp["pos_dec"][st], wl.L + wl.T + st, self.o_dec[st], self.lse_dec[st], self.wsd)
+            if ev:
+                ev["dec_call"][st][1].record()
+        if ev:
+            s.star_set_trace_events(None, None)
+
+
+def _ev():
+    return torch.cuda.Event(enable_timing=True)
+
+
+def _pair():
+    return (_ev(), _ev())
+
+
+def run_star(args, rank, world, local_rank):
+    import torch.distributed as dist
+    peaks = load_peaks()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl0 = get_config(args.config)
+    wl = dataclasses.replace(wl0, seed=wl0.seed + rank)
+    run = StarRun(wl, dev)
+    star = run.star
+
+    for _ in range(max(3, args.warmup)):
+        run.step()
+    torch.cuda.synchronize()
+    if star.star_device_status() != 0:
+        raise RuntimeError("device error after warm-up")
+
+    K = args.steps
+    evs = [{"p1": _pair(), "p2": _pair(), "dec": [_pair() for _ in range(wl.S)],
+            "dec_call": [_pair() for _ in range(wl.S)]} for _ in range(K)]
+    t0, t1 = _ev(), _ev()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        t0.record()
+        for k in range(K):
+            run.step(evs[k])
+        t1.record()
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    status = star.star_device_status()
+    ms_total = t0.elapsed_time(t1)
+    ms_tensor = torch.tensor([ms_total], device=dev)
+    if world > 1:
+        dist.all_reduce(ms_tensor, op=dist.ReduceOp.MAX)
+    ms_step = float(ms_tensor.item()) / K
+
+    p1_ms = statistics.mean(e["p1"][0].elapsed_time(e["p1"][1]) for e in evs)
+    p2_ms = statistics.mean(e["p2"][0].elapsed_time(e["p2"][1]) for e in evs)
+    dec_kernel_ms = [e["dec"][s][0].elapsed_time(e["dec"][s][1]) for e in evs for s in range(wl.S)]
+    dec_call_ms = [e["dec_call"][s][0].elapsed_time(e["dec_call"][s][1]) for e in evs for s in range(wl.S)]
+    flops = wl.phase1_flops()
+    tflops = flops / (p1_ms * 1e-3) / 1e12
+    dec_bytes = statistics.mean(wl.kv_bytes(wl.L + wl.T + s + 1) for s in range(wl.S))
+    dec_gbs = dec_bytes / (statistics.mean(dec_kernel_ms) * 1e-3) / 1e9
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(run, K, max(3, args.warmup), world)
+
+    value = world * wl.B * wl.L / (ms_step * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": max(3, args.warmup),
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16; 1% of context key rows x8 where the workload says peaky)",
+        "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d, "L": wl.L, "b": wl.b,
+                   "n": wl.n, "T": wl.T, "S": wl.S, "page_tokens": wl.page_tokens,
+                   "parallelism": f"independent sequences per GPU x{world}",
+                   "l2": "inputs larger than L2 (no flush)"},
+        "phase1": {"attn_ms": p1_ms, "ctx_tok_s": wl.B * wl.L / (p1_ms * 1e-3), "tflops": tflops,
+                   "frac_bf16_burst": tflops / peaks["bf16"], "frac_bf16_sustained": tflops / peaks["bf16_sustained"]},
+        "phase2": {"attn_ms": p2_ms},
+        "decode": {"us_per_step": 1e3 * statistics.mean(dec_call_ms), "kernel_us": 1e3 * statistics.mean(dec_kernel_ms),
+                   "bytes_per_step": dec_bytes, "kernel_gbs": dec_gbs, "frac_hbm": dec_gbs / peaks["hbm_gbs"]},
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
+                     "frac": tflops / peaks["bf16_sustained"], "traffic": None,
+                     "kernel": f"star_attn_kernel<{wl.d},0> (Phase 1)", "flop_per_launch": flops,
+                     "peak_source": peaks["kind"] + " bf16 sustained"},
+        "gpu_launches": run.launches_per_step * K,
+        "device_status": status,
+    }
+    if e2e:
+        line["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(run, args.cpu_rows)
+    if rank == 0:
+        line["clocks"] = clk.summary()
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(run, K, W, world):
+    """The same step with inputs in pinned host memory and results copied back, timed end to end."""
+    import torch.distributed as dist
+    wl, inp = run.wl, run.inp
+    names = ["q_ctx", "k_ctx", "v_ctx", "pos_ctx", "q_query", "k_query", "v_query", "pos_query",
+             "q_dec", "k_dec", "v_dec", "pos_dec"]
+    host_in = {n: inp[n].cpu().pin_memory() for n in names}
+    outs = [run.o_ctx, run.o_q, run.lse_q, run.o_dec, run.lse_dec]
+    host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+
+    def one():
+        for n in names:
+            inp[n].copy_(host_in[n], non_blocking=True)
+        run.step()
+        for o, h in zip(outs, host_out):
+            h.copy_(o, non_blocking=True)
+
+    for _ in range(W):
+        one()
+    torch.cuda.synchronize()
+    t0, t1 = _ev(), _ev()
+    if world > 1:
+        dist.barrier()
+    t0.record()
+    for _ in range(K):
+        one()
+    t1.record()
+    torch.cuda.synchronize()
+    ms = torch.tensor([t0.elapsed_time(t1) / K], device=run.dev)
+    if world > 1:
+        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
+    return {"value": world * wl.B * wl.L / (float(ms.item()) * 1e-3), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": float(ms.item())}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing
+# ---------------------------------------------------------------------------
+def _blas_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max((i.get("num_threads", 1) for i in info), default=1)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_phase1_sample(wl, host, blocks, rows_per_block, seed=0):
+    """Time the oracle's Phase-1 rows on a sample: `rows_per_block` rows of each listed block."""
+    import numpy as np
+    import oracle
+    rng = np.random.default_rng(seed)
+    rows = np.concatenate([i * wl.b + rng.choice(wl.b, rows_per_block, replace=False) for i in blocks])
+    rows.sort()
+    k = host["k"].float().numpy().astype(np.float64)
+    v = host["v"].float().numpy().astype(np.float64)
+    q = host["q"][rows].float().numpy().astype(np.float64)
+    pos = host["pos"].numpy().astype(np.int64)
+    t = time.perf_counter()
+    oracle.phase1_rows(rows, q, k, v, pos, wl.b, wl.theta)
+    return len(rows), time.perf_counter() - t
+
+
+def _host_seq0(inp):
+    return {"q": inp["q_ctx"][0].cpu(), "k": inp["k_ctx"][0].cpu(), "v": inp["v_ctx"][0].cpu(),
+            "pos": inp["pos_ctx"][0].cpu()}
+
+
+def cpu_baseline(run, rows_per_block):
+    wl = run.wl
+    host = _host_seq0(run.inp)
+    nrows, sec = oracle_phase1_sample(wl, host, range(wl.n), rows_per_block)
+    return {"value": nrows / sec, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"float64 oracle, Phase-1 output of {nrows} context rows ({rows_per_block} per block, all "
+                      f"{wl.Hq} heads, sequence 0) of {wl.name}; value = rows/s; {sec:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    wl = get_config(args.config)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = make_inputs(wl, dev, parts=("ctx",))
+    host = _host_seq0(inp)
+    del inp
+    rows_per_block = 4
+    W = max(3, args.warmup)
+    for w in range(W):
+        oracle_phase1_sample(wl, host, [w % wl.n], rows_per_block, seed=w)
+    tot_rows, tot_sec = 0, 0.0
+    for k in range(args.steps):
+        r, s = oracle_phase1_sample(wl, host, [k % wl.n], rows_per_block, seed=100 + k)
+        tot_rows += r
+        tot_sec += s
+    value = tot_rows / tot_sec
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": W, "ms_per_step": 1e3 * tot_sec / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (same seeded inputs as the CUDA arm)",
+        "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d, "L": wl.L, "b": wl.b,
+                   "n": wl.n, "T": wl.T, "S": wl.S},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+                         "sample": f"each step: float64 oracle Phase-1 output of {rows_per_block} context rows of one "
+                                   f"block (all {wl.Hq} heads) of {wl.name}; value = rows/s"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        run_star(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

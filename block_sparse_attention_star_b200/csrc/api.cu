@@ -1,0 +1,418 @@
+// C ABI of the Star Attention hot path: argument validation, workspace
+// planning and the launch sequence of each call.  See include/star.h.
+#include "star.h"
+#include "common.cuh"
+#include "internal.h"
+
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+thread_local cudaEvent_t g_trace_start = nullptr;
+thread_local cudaEvent_t g_trace_stop = nullptr;
+
+void trace_begin(cudaStream_t st) {
+  if (g_trace_start) cudaEventRecord(g_trace_start, st);
+}
+void trace_end(cudaStream_t st) {
+  if (g_trace_stop) cudaEventRecord(g_trace_stop, st);
+}
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(STAR_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+int num_sms() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+  return sms > 0 ? sms : 148;
+}
+
+int check_shape(const star_shape* s) {
+  if (!s) return fail(STAR_ERR_INVALID_ARG, "shape is NULL");
+  if (s->B <= 0 || s->Hq <= 0 || s->Hkv <= 0 || s->d <= 0 || s->L <= 0 || s->b <= 0 || s->n <= 0 ||
+      s->T_max < 0 || s->page_tokens <= 0)
+    return fail(STAR_ERR_INVALID_ARG, "shape fields must be positive (B=%d Hq=%d Hkv=%d d=%d L=%d b=%d n=%d T_max=%d P=%d)",
+                s->B, s->Hq, s->Hkv, s->d, s->L, s->b, s->n, s->T_max, s->page_tokens);
+  if (!(s->rope_theta > 0.0) || !std::isfinite(s->rope_theta))
+    return fail(STAR_ERR_INVALID_ARG, "rope_theta must be positive and finite");
+  if (s->Hq % s->Hkv) return fail(STAR_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", s->Hq, s->Hkv);
+  const int G = s->Hq / s->Hkv;
+  if (G != 2 && G != 4 && G != 8)
+    return fail(STAR_ERR_UNSUPPORTED_SHAPE, "GQA group size Hq/Hkv = %d is not supported (2, 4 or 8)", G);
+  if (s->d != 64 && s->d != 128) return fail(STAR_ERR_UNSUPPORTED_SHAPE, "head dim %d is not supported (64 or 128)", s->d);
+  if ((int64_t)s->n * s->b != s->L)
+    return fail(STAR_ERR_UNSUPPORTED_SHAPE, "L (%d) must equal n*b (%d*%d): ragged last blocks are not supported",
+                s->L, s->n, s->b);
+  if (s->b % 128) return fail(STAR_ERR_UNSUPPORTED_SHAPE, "block size b (%d) must be a multiple of 128", s->b);
+  if (s->page_tokens % 128) return fail(STAR_ERR_UNSUPPORTED_SHAPE, "page_tokens (%d) must be a multiple of 128", s->page_tokens);
+  if (s->b % s->page_tokens)
+    return fail(STAR_ERR_UNSUPPORTED_SHAPE, "b (%d) must be a multiple of page_tokens (%d)", s->b, s->page_tokens);
+  if ((int64_t)s->L + round_up(s->T_max, 128) >= (int64_t)1 << 30)
+    return fail(STAR_ERR_UNSUPPORTED_SHAPE, "L + T_max too large");
+  return STAR_OK;
+}
+
+int64_t pages_needed(const star_shape* s) {
+  return ((int64_t)s->L + round_up(s->T_max, 128) + s->page_tokens - 1) / s->page_tokens;
+}
+
+int check_cache(const star_shape* s, const star_cache* c) {
+  if (!c) return fail(STAR_ERR_INVALID_ARG, "cache is NULL");
+  if (!c->k_pool || !c->v_pool || !c->page_table) return fail(STAR_ERR_INVALID_ARG, "cache pointers must be non-NULL");
+  if (!aligned16(c->k_pool) || !aligned16(c->v_pool) || !aligned16(c->page_table))
+    return fail(STAR_ERR_ALIGNMENT, "cache pointers must be 16-byte aligned");
+  if (c->max_pages < pages_needed(s))
+    return fail(STAR_ERR_CAPACITY, "page table has %d pages per sequence, %lld needed", c->max_pages,
+                (long long)pages_needed(s));
+  if (c->num_pages <= 0) return fail(STAR_ERR_CAPACITY, "num_pages must be positive");
+  return STAR_OK;
+}
+
+star::CacheView view(const star_shape* s, const star_cache* c) {
+  star::CacheView v;
+  v.k_pool = c->k_pool;
+  v.v_pool = c->v_pool;
+  v.page_table = c->page_table;
+  v.max_pages = c->max_pages;
+  v.num_pages = c->num_pages;
+  v.P = s->page_tokens;
+  return v;
+}
+
+star::RopeTable rope_table(const star_shape* s) {
+  star::RopeTable t;
+  for (int j = 0; j < star::kMaxHalfDimHost; ++j)
+    t.inv_freq[j] = j < s->d / 2 ? std::pow(s->rope_theta, -2.0 * j / s->d) : 0.0;
+  return t;
+}
+
+float scale_log2(const star_shape* s) { return (float)(1.4426950408889634 / std::sqrt((double)s->d)); }
+
+#define STAR_REQUIRE_PTR(p, name)                                                    \
+  do {                                                                               \
+    if (!(p)) return fail(STAR_ERR_INVALID_ARG, "%s is NULL", name);                 \
+    if (!aligned16(p)) return fail(STAR_ERR_ALIGNMENT, "%s is not 16-byte aligned", name); \
+  } while (0)
+
+// Phase 2 splits each block into chunks_per_block parts so the grid fills the
+// GPU; the smallest divisor of b/128 that gives >= 2 items per SM.
+int phase2_chunks_per_block(const star_shape* s, int T) {
+  const int G = s->Hq / s->Hkv;
+  int TQ = 1;
+  while (TQ < T && TQ < 128) TQ <<= 1;
+  const int HT = 128 / TQ;
+  const int NTT = (T + TQ - 1) / TQ;
+  const int NHT = (G + HT - 1) / HT;
+  const int npairs = (NTT * NHT + 1) / 2;
+  const int64_t base = (int64_t)s->n * s->B * s->Hkv * npairs;
+  const int64_t need = (2LL * num_sms() + base - 1) / base;
+  const int nb = s->b / 128;
+  for (int c = 1; c <= nb; ++c)
+    if (nb % c == 0 && c >= need) return c;
+  return nb;
+}
+
+size_t phase2_ws_bytes(const star_shape* s, int T) {
+  const int cpb = phase2_chunks_per_block(s, T);
+  if (cpb == 1) return 0;
+  const size_t rows = (size_t)s->B * T * s->Hq;
+  const size_t parts = (size_t)s->n * cpb;
+  return round_up(parts * rows * s->d * sizeof(float), 256) + round_up(parts * rows * sizeof(float), 256);
+}
+
+int decode_chunk(const star_shape* s) {
+  return star::decode_pick_chunk(s->B, s->Hkv, s->Hq / s->Hkv, s->L + s->T_max, num_sms());
+}
+
+size_t decode_ws_bytes(const star_shape* s) {
+  const int chunk = decode_chunk(s);
+  const size_t nch = (size_t)star::decode_num_chunks(s->L + s->T_max, chunk);
+  const size_t rows = (size_t)s->B * s->Hq;
+  return round_up(nch * rows * s->d * sizeof(float), 256) + round_up(nch * rows * sizeof(float), 256);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* star_version(void) { return "star-b200 0.1 (sm_100a)"; }
+
+const char* star_last_error(void) { return g_last_error; }
+
+int star_pages_needed(const star_shape* shape, int32_t* max_pages_out) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (!max_pages_out) return fail(STAR_ERR_INVALID_ARG, "max_pages_out is NULL");
+  *max_pages_out = (int32_t)pages_needed(shape);
+  return STAR_OK;
+}
+
+int star_page_table_fill(const star_shape* shape, int32_t* page_table_host, int32_t max_pages, int32_t first_page) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (!page_table_host) return fail(STAR_ERR_INVALID_ARG, "page_table_host is NULL");
+  if (max_pages < pages_needed(shape))
+    return fail(STAR_ERR_CAPACITY, "max_pages %d < %lld needed", max_pages, (long long)pages_needed(shape));
+  if (first_page < 0) return fail(STAR_ERR_INVALID_ARG, "first_page must be >= 0");
+  for (int64_t s = 0; s < shape->B; ++s)
+    for (int64_t j = 0; j < max_pages; ++j) page_table_host[s * max_pages + j] = (int32_t)(first_page + s * max_pages + j);
+  return STAR_OK;
+}
+
+int star_workspace_size(const star_shape* shape, int op, int32_t T, size_t* bytes_out) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (!bytes_out) return fail(STAR_ERR_INVALID_ARG, "bytes_out is NULL");
+  switch (op) {
+    case STAR_OP_PHASE1: *bytes_out = 0; return STAR_OK;
+    case STAR_OP_PHASE2:
+      if (T <= 0 || T > shape->T_max) return fail(STAR_ERR_INVALID_ARG, "T (%d) must be in [1, T_max=%d]", T, shape->T_max);
+      *bytes_out = phase2_ws_bytes(shape, T);
+      return STAR_OK;
+    case STAR_OP_DECODE: *bytes_out = decode_ws_bytes(shape); return STAR_OK;
+    default: return fail(STAR_ERR_INVALID_ARG, "unknown op %d", op);
+  }
+}
+
+int star_build_positions(const star_shape* shape, const star_cache* cache, const int32_t* pos_ctx, int32_t* aug_pos,
+                         int32_t* block_map, star_stream_t stream) {
+  int rc = check_shape(shape);
+  if (!rc) rc = check_cache(shape, cache);
+  if (rc) return rc;
+  STAR_REQUIRE_PTR(pos_ctx, "pos_ctx");
+  STAR_REQUIRE_PTR(aug_pos, "aug_pos");
+  STAR_REQUIRE_PTR(block_map, "block_map");
+  cudaError_t e = star::launch_build_positions(pos_ctx, shape->B, shape->L, shape->b, view(shape, cache), aug_pos,
+                                               block_map, (cudaStream_t)stream);
+  return e == cudaSuccess ? STAR_OK : cuda_fail(e, "build_positions launch");
+}
+
+int star_kv_append(const star_shape* shape, const star_cache* cache, const void* k, const void* v, const int32_t* pos,
+                   int32_t start, int32_t ntok, star_stream_t stream) {
+  int rc = check_shape(shape);
+  if (!rc) rc = check_cache(shape, cache);
+  if (rc) return rc;
+  STAR_REQUIRE_PTR(k, "k");
+  STAR_REQUIRE_PTR(v, "v");
+  STAR_REQUIRE_PTR(pos, "pos");
+  if (start < 0 || ntok < 0) return fail(STAR_ERR_INVALID_ARG, "start and ntok must be >= 0");
+  if ((int64_t)start + ntok > (int64_t)shape->L + shape->T_max)
+    return fail(STAR_ERR_CAPACITY, "slots [%d, %d) exceed L + T_max = %d", start, start + ntok, shape->L + shape->T_max);
+  cudaError_t e = star::launch_rope_append(k, v, pos, shape->B, ntok, start, shape->Hkv, shape->d, view(shape, cache),
+                                           rope_table(shape), (cudaStream_t)stream);
+  return e == cudaSuccess ? STAR_OK : cuda_fail(e, "kv_append launch");
+}
+
+int star_phase1_encode(const star_shape* shape, const star_cache* cache, const void* q, const void* k, const void* v,
+                       const int32_t* pos_ctx, void* out, void* ws, size_t ws_bytes, star_stream_t stream) {
+  (void)ws;
+  (void)ws_bytes;
+  int rc = check_shape(shape);
+  if (!rc) rc = check_cache(shape, cache);
+  if (rc) return rc;
+  STAR_REQUIRE_PTR(q, "q");
+  STAR_REQUIRE_PTR(k, "k");
+  STAR_REQUIRE_PTR(v, "v");
+  STAR_REQUIRE_PTR(pos_ctx, "pos_ctx");
+  STAR_REQUIRE_PTR(out, "out");
+  cudaStream_t st = (cudaStream_t)stream;
+  const star::CacheView cv = view(shape, cache);
+  const star::RopeTable rt = rope_table(shape);
+  cudaError_t e = star::launch_rope_append(k, v, pos_ctx, shape->B, shape->L, 0, shape->Hkv, shape->d, cv, rt, st);
+  if (e != cudaSuccess) return cuda_fail(e, "phase1 kv append");
+  e = star::launch_zero_slots(shape->B, shape->L, shape->L + (int)round_up(shape->T_max, 128), shape->Hkv, shape->d,
+                              cv, st);
+  if (e != cudaSuccess) return cuda_fail(e, "phase1 tail clear");
+  star::AttnLaunch a;
+  memset(&a, 0, sizeof(a));
+  a.mode = 0;
+  a.B = shape->B;
+  a.Hq = shape->Hq;
+  a.Hkv = shape->Hkv;
+  a.d = shape->d;
+  a.L = shape->L;
+  a.b = shape->b;
+  a.n = shape->n;
+  a.q = q;
+  a.q_pos = pos_ctx;
+  a.Ntok = shape->L;
+  a.cache = cv;
+  a.out_bf16 = out;
+  a.chunks_per_block = 1;
+  a.scale_log2 = scale_log2(shape);
+  a.rope = rt;
+  const char* why = nullptr;
+  trace_begin(st);
+  e = star::launch_attention(a, st, &why);
+  trace_end(st);
+  if (e != cudaSuccess) return why ? fail(STAR_ERR_CUDA, "%s", why) : cuda_fail(e, "phase1 attention launch");
+  return STAR_OK;
+}
+
+int star_phase2_partial(const star_shape* shape, const star_cache* cache, const void* q, const void* k, const void* v,
+                        const int32_t* q_pos, int32_t T, float* o_part, float* lse_part, void* ws, size_t ws_bytes,
+                        star_stream_t stream) {
+  int rc = check_shape(shape);
+  if (!rc) rc = check_cache(shape, cache);
+  if (rc) return rc;
+  STAR_REQUIRE_PTR(q, "q");
+  STAR_REQUIRE_PTR(q_pos, "q_pos");
+  STAR_REQUIRE_PTR(o_part, "o_part");
+  STAR_REQUIRE_PTR(lse_part, "lse_part");
+  if ((k == nullptr) != (v == nullptr)) return fail(STAR_ERR_INVALID_ARG, "k and v must both be given or both be NULL");
+  if (T <= 0 || T > shape->T_max) return fail(STAR_ERR_INVALID_ARG, "T (%d) must be in [1, T_max=%d]", T, shape->T_max);
+  const size_t need = phase2_ws_bytes(shape, T);
+  if (need > 0) {
+    STAR_REQUIRE_PTR(ws, "ws");
+    if (ws_bytes < need) return fail(STAR_ERR_CAPACITY, "workspace %zu bytes < %zu needed", ws_bytes, need);
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  const star::CacheView cv = view(shape, cache);
+  const star::RopeTable rt = rope_table(shape);
+  if (k) {
+    STAR_REQUIRE_PTR(k, "k");
+    STAR_REQUIRE_PTR(v, "v");
+    cudaError_t e = star::launch_rope_append(k, v, q_pos, shape->B, T, shape->L, shape->Hkv, shape->d, cv, rt, st);
+    if (e != cudaSuccess) return cuda_fail(e, "phase2 kv append");
+  }
+  const int cpb = phase2_chunks_per_block(shape, T);
+  const size_t rows = (size_t)shape->B * T * shape->Hq;
+  const size_t parts = (size_t)shape->n * cpb;
+  float* o_dst = o_part;
+  float* l_dst = lse_part;
+  if (cpb > 1) {
+    o_dst = reinterpret_cast<float*>(ws);
+    l_dst = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + round_up(parts * rows * shape->d * sizeof(float), 256));
+  }
+  star::AttnLaunch a;
+  memset(&a, 0, sizeof(a));
+  a.mode = 1;
+  a.B = shape->B;
+  a.Hq = shape->Hq;
+  a.Hkv = shape->Hkv;
+  a.d = shape->d;
+  a.L = shape->L;
+  a.b = shape->b;
+  a.n = shape->n;
+  a.q = q;
+  a.q_pos = q_pos;
+  a.Ntok = T;
+  a.cache = cv;
+  a.out_f32 = o_dst;
+  a.lse_f32 = l_dst;
+  a.chunks_per_block = cpb;
+  a.scale_log2 = scale_log2(shape);
+  a.rope = rt;
+  const char* why = nullptr;
+  trace_begin(st);
+  cudaError_t e = star::launch_attention(a, st, &why);
+  trace_end(st);
+  if (e != cudaSuccess) return why ? fail(STAR_ERR_CUDA, "%s", why) : cuda_fail(e, "phase2 attention launch");
+  if (cpb > 1) {
+    e = star::launch_lse_merge(shape->n, cpb, (int64_t)rows, shape->d, o_dst, l_dst, o_part, false, lse_part, st);
+    if (e != cudaSuccess) return cuda_fail(e, "phase2 chunk merge");
+  }
+  return STAR_OK;
+}
+
+int star_lse_merge(int32_t n_parts, int64_t rows, int32_t d, const float* o_part, const float* lse_part, void* out,
+                   float* lse_out, star_stream_t stream) {
+  if (n_parts <= 0 || rows < 0) return fail(STAR_ERR_INVALID_ARG, "n_parts must be > 0 and rows >= 0");
+  if (d != 64 && d != 128) return fail(STAR_ERR_UNSUPPORTED_SHAPE, "head dim %d is not supported (64 or 128)", d);
+  STAR_REQUIRE_PTR(o_part, "o_part");
+  STAR_REQUIRE_PTR(lse_part, "lse_part");
+  STAR_REQUIRE_PTR(out, "out");
+  if (lse_out && !aligned16(lse_out)) return fail(STAR_ERR_ALIGNMENT, "lse_out is not 16-byte aligned");
+  cudaError_t e = star::launch_lse_merge(1, n_parts, rows, d, o_part, lse_part, out, true, lse_out, (cudaStream_t)stream);
+  return e == cudaSuccess ? STAR_OK : cuda_fail(e, "lse_merge launch");
+}
+
+int star_decode_step(const star_shape* shape, const star_cache* cache, const void* q, const void* k, const void* v,
+                     const int32_t* pos, int32_t cur_len, void* out, float* lse_out, void* ws, size_t ws_bytes,
+                     star_stream_t stream) {
+  int rc = check_shape(shape);
+  if (!rc) rc = check_cache(shape, cache);
+  if (rc) return rc;
+  STAR_REQUIRE_PTR(q, "q");
+  STAR_REQUIRE_PTR(k, "k");
+  STAR_REQUIRE_PTR(v, "v");
+  STAR_REQUIRE_PTR(pos, "pos");
+  STAR_REQUIRE_PTR(out, "out");
+  STAR_REQUIRE_PTR(ws, "ws");
+  if (lse_out && !aligned16(lse_out)) return fail(STAR_ERR_ALIGNMENT, "lse_out is not 16-byte aligned");
+  if (cur_len < 0 || cur_len >= shape->L + shape->T_max)
+    return fail(STAR_ERR_CAPACITY, "cur_len %d outside [0, L + T_max = %d)", cur_len, shape->L + shape->T_max);
+  const size_t need = decode_ws_bytes(shape);
+  if (ws_bytes < need) return fail(STAR_ERR_CAPACITY, "workspace %zu bytes < %zu needed", ws_bytes, need);
+  cudaStream_t st = (cudaStream_t)stream;
+  const star::CacheView cv = view(shape, cache);
+  const star::RopeTable rt = rope_table(shape);
+  cudaError_t e = star::launch_rope_append(k, v, pos, shape->B, 1, cur_len, shape->Hkv, shape->d, cv, rt, st);
+  if (e != cudaSuccess) return cuda_fail(e, "decode kv append");
+  const int chunk = decode_chunk(shape);
+  const int n_keys = cur_len + 1;
+  const int nch = star::decode_num_chunks(n_keys, chunk);
+  const size_t rows = (size_t)shape->B * shape->Hq;
+  const size_t nch_max = (size_t)star::decode_num_chunks(shape->L + shape->T_max, chunk);
+  star::DecodeLaunch a;
+  a.B = shape->B;
+  a.Hq = shape->Hq;
+  a.Hkv = shape->Hkv;
+  a.d = shape->d;
+  a.q = q;
+  a.pos = pos;
+  a.n_keys = n_keys;
+  a.chunk = chunk;
+  a.cache = cv;
+  a.o_ws = reinterpret_cast<float*>(ws);
+  a.lse_ws = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + round_up(nch_max * rows * shape->d * sizeof(float), 256));
+  a.scale_log2 = scale_log2(shape);
+  a.rope = rt;
+  trace_begin(st);
+  e = star::launch_decode(a, st);
+  trace_end(st);
+  if (e != cudaSuccess) return cuda_fail(e, "decode attention launch");
+  e = star::launch_lse_merge(1, nch, (int64_t)rows, shape->d, a.o_ws, a.lse_ws, out, true, lse_out, st);
+  return e == cudaSuccess ? STAR_OK : cuda_fail(e, "decode merge launch");
+}
+
+int star_set_trace_events(void* start_event, void* stop_event) {
+  if ((start_event == nullptr) != (stop_event == nullptr))
+    return fail(STAR_ERR_INVALID_ARG, "trace events must both be given or both be NULL");
+  g_trace_start = reinterpret_cast<cudaEvent_t>(start_event);
+  g_trace_stop = reinterpret_cast<cudaEvent_t>(stop_event);
+  return STAR_OK;
+}
+
+int star_device_status(star_stream_t stream, int32_t* status_out) {
+  int code = 0;
+  cudaError_t e = star::read_and_clear_device_error(&code, (cudaStream_t)stream);
+  if (status_out) *status_out = code;
+  if (e != cudaSuccess) return cuda_fail(e, "device status");
+  if (code == star::kDevBadPage) return fail(STAR_ERR_CAPACITY, "a page-table entry was outside [0, num_pages)");
+  if (code != 0) return fail(STAR_ERR_TIMEOUT, "a kernel gave up a bounded wait (code %d)", code);
+  return STAR_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,674 @@
+// Star Attention tensor-core attention for sm_100a (tcgen05 + TMEM + TMA).
+//
+// One kernel serves two steps of the hot path:
+//
+//  * mode 0 -- Phase 1, anchor-augmented blockwise-local causal attention
+//    ("Star Attention 完全拆解(一)", Phase 1: "被增广的上下文" and "局部注意力与
+//    KV 丢弃").  Query row t of block i > 1 attends to the anchor keys [0, b)
+//    and to its own block's keys up to itself; block 1 is plain causal.  The
+//    anchor is never materialised: its keys are block 1's cached pages (the
+//    anchor keeps block 1's positions, so its roped K/V equal block 1's bit for
+//    bit), and anchor rows are never recomputed (their outputs are discarded).
+//  * mode 1 -- Phase 2, the query tokens' local attention against each block
+//    ("Phase 2: 局部注意力与本地统计量"), written as per-part (O, LSE) partials
+//    for the exact log-sum-exp merge ("组装全局结果", "数值稳定性").  A part is a
+//    chunk of one block; the last block's last chunk also covers the query tail.
+//
+// Both are "causal by cache index over a key set": a work item lists up to two
+// runs of 128-key tiles, and a key is visible to a row iff its cache index is
+// <= the row's cache index.
+//
+// CTA organisation (384 threads, persistent, one CTA per SM):
+//   warp 0      TMA producer: K and V tiles from the paged cache into two
+//               shared-memory rings (128-byte swizzle, no multicast).
+//   warp 1      MMA issuer: S_w = Q_w K^T (SS form) and O_w += P_w V (A from TMEM).
+//   warps 4-7   softmax warpgroup 0 (Q tile 0: rows <-> TMEM lanes 0..127)
+//   warps 8-11  softmax warpgroup 1 (Q tile 1)
+// The two Q tiles of an item share every K/V tile (two heads of one GQA group in
+// Phase 1; two row tiles of the group in Phase 2), so each K/V byte staged in
+// shared memory feeds 2 x 128 query rows.  While warpgroup 0 turns S_0 into
+// P_0 the tensor core runs warpgroup 1's products, and vice versa.
+//
+// TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+d), O_1 [384,384+d).
+// P_w (bf16, two per 32-bit column) overwrites the first 64 columns of S_w.
+// Softmax uses the online (running max m, running sum l) formulation of the
+// FlashAttention section of the long-context attention review, in base 2 with a
+// lazily updated max: O and l are rescaled only when the tile max exceeds the
+// running max by more than 8 (so P <= 256 always fits bf16 and f32 sums).
+#include "common.cuh"
+#include "internal.h"
+
+#include <algorithm>
+#include <climits>
+#include <cstring>
+
+namespace star {
+
+__device__ int g_device_error = 0;
+
+namespace {
+
+constexpr int kThreads = 384;
+constexpr int kRows = 128;        // rows per Q tile (UMMA M)
+constexpr int kKeys = 128;        // keys per K/V tile (UMMA N of QK^T, K of PV)
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;
+
+struct Params {
+  const bf16* q;
+  const int32_t* q_pos;
+  bf16* out_bf16;
+  float* out_f32;
+  float* lse_f32;
+  const int32_t* page_table;
+  int max_pages, num_pages, P;
+  int B, Hq, Hkv, G, L, b, n, Ntok;
+  // Phase-2 tiling
+  int chunk_keys, chunks_per_block, tail_tiles, TQ, HT, NTT, NHT, npairs;
+  int num_items;
+  float scale_log2;
+  double inv_freq[kMaxHalfDim];
+};
+
+struct Item {
+  int bi, g;
+  int a_start, a_tiles;   // first run of key tiles (cache index of its first key, tile count)
+  int b_start, b_tiles;   // second run
+  int part;               // Phase 2: output part (global chunk index)
+  int r0;                 // Phase 1: context index of the tile's first row
+  int hp;                 // Phase 1: head pair in the group; Phase 2: row-tile pair
+};
+
+// Work items.  Phase 1, per (sequence, KV head): items of blocks 2..n first,
+// then block 1's, each run ordered by descending q-tile, so item cost falls
+// monotonically and the round-robin assignment to CTAs stays balanced.
+template <int MODE>
+__device__ __forceinline__ Item decode_item(const Params& p, int idx) {
+  Item it;
+  if (MODE == 0) {
+    const int nqt = p.b / kRows;
+    const int npairs = p.G / 2;
+    const int per_group = p.n * nqt * npairs;
+    const int grp = idx / per_group;
+    int w = idx - grp * per_group;
+    it.bi = grp / p.Hkv;
+    it.g = grp - it.bi * p.Hkv;
+    const int nonanchor = (p.n - 1) * nqt * npairs;
+    int t, i;
+    if (w < nonanchor) {
+      const int per_t = (p.n - 1) * npairs;
+      t = nqt - 1 - w / per_t;
+      const int rem = w - (w / per_t) * per_t;
+      i = 1 + rem / npairs;
+      it.hp = rem - (rem / npairs) * npairs;
+    } else {
+      w -= nonanchor;
+      t = nqt - 1 - w / npairs;
+      i = 0;
+      it.hp = w - (w / npairs) * npairs;
+    }
+    it.a_start = 0;
+    it.a_tiles = (i > 0) ? nqt : 0;
+    it.b_start = i * p.b;
+    it.b_tiles = t + 1;
+    it.part = i;
+    it.r0 = i * p.b + t * kRows;
+  } else {
+    it.hp = idx % p.npairs;
+    int rest = idx / p.npairs;
+    it.g = rest % p.Hkv;
+    rest /= p.Hkv;
+    it.bi = rest % p.B;
+    const int c = rest / p.B;
+    it.part = c;
+    it.a_start = c * p.chunk_keys;
+    it.a_tiles = p.chunk_keys / kKeys;
+    const bool last = (c == p.n * p.chunks_per_block - 1);
+    it.b_start = p.L;
+    it.b_tiles = last ? p.tail_tiles : 0;
+    it.r0 = 0;
+  }
+  return it;
+}
+
+__device__ __forceinline__ int tile_key0(const Item& it, int j) {
+  return j < it.a_tiles ? it.a_start + j * kKeys : it.b_start + (j - it.a_tiles) * kKeys;
+}
+
+struct RowInfo {
+  bool valid;
+  int head;       // query head
+  int tok;        // index into q / q_pos / outputs
+  int cache_idx;  // cache index used by the causal rule
+  int pos;        // RoPE position
+};
+
+template <int MODE>
+__device__ __forceinline__ RowInfo row_info(const Params& p, const Item& it, int wg, int row) {
+  RowInfo r;
+  if (MODE == 0) {
+    r.valid = true;
+    r.head = it.g * p.G + 2 * it.hp + wg;
+    r.tok = it.r0 + row;
+    r.cache_idx = r.tok;
+  } else {
+    const int rt = 2 * it.hp + wg;
+    const int ht = rt / p.NTT, tt = rt - (rt / p.NTT) * p.NTT;
+    const int hl = ht * p.HT + row / p.TQ;
+    const int t = tt * p.TQ + (row % p.TQ);
+    r.valid = (rt < p.NTT * p.NHT) && (hl < p.G) && (t < p.Ntok);
+    r.head = it.g * p.G + (r.valid ? hl : 0);
+    r.tok = r.valid ? t : 0;
+    r.cache_idx = r.valid ? p.L + t : INT_MAX;
+  }
+  r.pos = r.valid ? p.q_pos[(size_t)it.bi * p.Ntok + r.tok] : 0;
+  if (!r.valid) r.cache_idx = INT_MAX;
+  return r;
+}
+
+// One thread writes its Q row, rotated and rounded to bf16, into the K-major
+// 128-byte-swizzled tile: element (row, col) lives in the 64-column atom col/64
+// at byte row*128 + 16*((col%64/8) ^ (row%8)) + 2*(col%8).
+template <int D>
+__device__ __forceinline__ void load_q_row(const Params& p, const Item& it, const RowInfo& r, uint8_t* sQ, int row) {
+  constexpr int H2 = D / 2;
+  const bf16* src = p.q + (((size_t)it.bi * p.Ntok + r.tok) * p.Hq + r.head) * D;
+#pragma unroll
+  for (int c = 0; c < D / 16; ++c) {
+    uint4 a = make_uint4(0, 0, 0, 0), bq = make_uint4(0, 0, 0, 0);
+    if (r.valid) {
+      a = __ldg(reinterpret_cast<const uint4*>(src + 8 * c));
+      bq = __ldg(reinterpret_cast<const uint4*>(src + H2 + 8 * c));
+    }
+    const uint32_t* aw = reinterpret_cast<const uint32_t*>(&a);
+    const uint32_t* bw = reinterpret_cast<const uint32_t*>(&bq);
+    uint32_t lo[4], hi[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 x1 = unpack_bf16x2(aw[e]);
+      const float2 x2 = unpack_bf16x2(bw[e]);
+      float c0, s0, c1, s1;
+      rope_sincos(r.pos, p.inv_freq[8 * c + 2 * e], c0, s0);
+      rope_sincos(r.pos, p.inv_freq[8 * c + 2 * e + 1], c1, s1);
+      lo[e] = pack_bf16x2(x1.x * c0 - x2.x * s0, x1.y * c1 - x2.y * s1);
+      hi[e] = pack_bf16x2(x2.x * c0 + x1.x * s0, x2.y * c1 + x1.y * s1);
+    }
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int col = half * H2 + 8 * c;
+      const int atom = col / 64;
+      const int chunk = (col % 64) / 8;
+      uint8_t* dst = sQ + atom * (kRows * 128) + row * 128 + ((chunk ^ (row & 7)) * 16);
+      const uint32_t* w = half ? hi : lo;
+      *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+}
+
+template <int D, int MODE, int NSK, int NSV>
+struct Smem {
+  static constexpr int kTile = kRows * D * 2;  // bytes of one 128 x D bf16 tile
+  static constexpr int kQ0 = 0;
+  static constexpr int kK = 2 * kTile;
+  static constexpr int kV = kK + NSK * kTile;
+  static constexpr int kBar = kV + NSV * kTile;
+  static constexpr int kNumBars = 2 * NSK + 2 * NSV + 4 * 2 + 1;
+  static constexpr int kTmemSlot = kBar + kNumBars * 8;
+  static constexpr int kEnd = kTmemSlot + 16;
+  static constexpr int kBytes = kEnd + 1024;  // slack for 1024-byte alignment
+};
+
+template <int D, int MODE, int NSK, int NSV>
+__global__ void __launch_bounds__(kThreads, 1)
+    star_attn_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                     const __grid_constant__ Params p) {
+  using S = Smem<D, MODE, NSK, NSV>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
+  uint64_t* k_full = bars;
+  uint64_t* k_empty = k_full + NSK;
+  uint64_t* v_full = k_empty + NSK;
+  uint64_t* v_empty = v_full + NSV;
+  uint64_t* q_full = v_empty + NSV;   // [2]
+  uint64_t* s_full = q_full + 2;      // [2]
+  uint64_t* p_full = s_full + 2;      // [2]
+  uint64_t* o_full = p_full + 2;      // [2]
+  uint64_t* drain = o_full + 2;       // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kTmemSlot);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NSK; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1); }
+    for (int s = 0; s < NSV; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1); }
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(&q_full[w], kRows);
+      mbar_init(&s_full[w], 1);
+      mbar_init(&p_full[w], kRows);
+      mbar_init(&o_full[w], 1);
+    }
+    mbar_init(drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t kcnt = 0, vcnt = 0;
+      bool ok = true;
+      for (int idx = blockIdx.x; idx < p.num_items && ok; idx += gridDim.x) {
+        const Item it = decode_item<MODE>(p, idx);
+        const int nt = it.a_tiles + it.b_tiles;
+        for (int j = 0; j < nt && ok; ++j) {
+          const int k0 = tile_key0(it, j);
+          int page = p.page_table[(size_t)it.bi * p.max_pages + k0 / p.P];
+          if (page < 0 || page >= p.num_pages) { record_error(kDevBadPage); page = 0; }
+          const int slot = k0 % p.P;
+          {
+            const int s = kcnt % NSK;
+            ok = mbar_wait(&k_empty[s], ((kcnt / NSK) & 1) ^ 1, kDevTimeoutProducer);
+            if (!ok) break;
+            mbar_arrive_expect_tx(&k_full[s], S::kTile);
+            uint8_t* dst = smem + S::kK + s * S::kTile;
+#pragma unroll
+            for (int h = 0; h < D / 64; ++h)
+              tma_load_4d(dst + h * (kKeys * 128), &tmK, &k_full[s], h * 64, slot, it.g, page);
+            ++kcnt;
+          }
+          {
+            const int s = vcnt % NSV;
+            ok = mbar_wait(&v_empty[s], ((vcnt / NSV) & 1) ^ 1, kDevTimeoutProducer);
+            if (!ok) break;
+            mbar_arrive_expect_tx(&v_full[s], S::kTile);
+            uint8_t* dst = smem + S::kV + s * S::kTile;
+#pragma unroll
+            for (int h = 0; h < D / 64; ++h)
+              tma_load_4d(dst + h * (kKeys * 128), &tmV, &v_full[s], h * 64, slot, it.g, page);
+            ++vcnt;
+          }
+        }
+      }
+      // Drain: every load issued into a stage has landed before the CTA exits.
+      for (uint32_t s = 0; s < NSK && s < kcnt; ++s) {
+        const uint32_t last = kcnt - 1 - ((kcnt - 1 - s) % NSK);
+        mbar_wait(&k_full[s], (last / NSK) & 1, kDevTimeoutProducer);
+      }
+      for (uint32_t s = 0; s < NSV && s < vcnt; ++s) {
+        const uint32_t last = vcnt - 1 - ((vcnt - 1 - s) % NSV);
+        mbar_wait(&v_full[s], (last / NSV) & 1, kDevTimeoutProducer);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = umma_idesc_bf16(kRows, kKeys, 0, 0);
+      constexpr uint32_t idesc_pv = umma_idesc_bf16(kRows, D, 0, 1);
+      const uint32_t sQ = smem_u32(smem + S::kQ0);
+      const uint32_t sK = smem_u32(smem + S::kK);
+      const uint32_t sV = smem_u32(smem + S::kV);
+      uint32_t kcnt = 0, vcnt = 0, qph = 0, pph[2] = {0, 0};
+      bool ok = true;
+      bool issued = false;
+
+      // S_w = Q_w K^T: K-major A and B, 128-byte swizzle, 8-row groups 1024 B apart;
+      // a 16-element K step is 32 B inside a 64-column atom, atoms are 16 KB apart.
+      auto issue_s = [&](int w, int ks) {
+        const uint32_t qa = sQ + w * S::kTile;
+        const uint32_t kb = sK + ks * S::kTile;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * (kRows * 128) + (kk % 4) * 32;
+          mma_ss(tbase + w * 128, umma_desc_sw128(qa + off, 16, 1024), umma_desc_sw128(kb + off, 16, 1024),
+                 idesc_qk, kk > 0 ? 1u : 0u);
+        }
+      };
+      // O_w += P_w V: P from TMEM (8 columns per 16 keys); V MN-major (d contiguous),
+      // 8 keys of 128 B per swizzle group (SBO 1024 B), 64-column d atoms 16 KB apart (LBO).
+      auto issue_pv = [&](int w, int vs, bool acc) {
+        const uint32_t vb = sV + vs * S::kTile;
+#pragma unroll
+        for (int kk = 0; kk < kKeys / 16; ++kk) {
+          mma_ts(tbase + 256 + w * 128, tbase + w * 128 + kk * 8, umma_desc_sw128(vb + kk * 2048, kKeys * 128, 1024),
+                 idesc_pv, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+
+      for (int idx = blockIdx.x; idx < p.num_items && ok; idx += gridDim.x) {
+        const Item it = decode_item<MODE>(p, idx);
+        const int nt = it.a_tiles + it.b_tiles;
+        ok = mbar_wait(&q_full[0], qph, kDevTimeoutMma) && mbar_wait(&q_full[1], qph, kDevTimeoutMma);
+        if (!ok) break;
+        qph ^= 1;
+        tc_fence_after();
+        for (int j = 0; j < nt; ++j) {
+          const int ks = kcnt % NSK;
+          ok = mbar_wait(&k_full[ks], (kcnt / NSK) & 1, kDevTimeoutMma);
+          if (!ok) break;
+          tc_fence_after();
+          int vs = 0;
+          if (j > 0) {
+            ok = mbar_wait(&p_full[0], pph[0], kDevTimeoutMma);
+            if (!ok) break;
+            pph[0] ^= 1;
+            vs = vcnt % NSV;
+            ok = mbar_wait(&v_full[vs], (vcnt / NSV) & 1, kDevTimeoutMma);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(0, vs, j > 1);
+          }
+          issue_s(0, ks);
+          issued = true;
+          mma_commit(&s_full[0]);
+          if (j > 0) {
+            ok = mbar_wait(&p_full[1], pph[1], kDevTimeoutMma);
+            if (!ok) break;
+            pph[1] ^= 1;
+            tc_fence_after();
+            issue_pv(1, vs, j > 1);
+            mma_commit(&v_empty[vs]);
+            ++vcnt;
+          }
+          issue_s(1, ks);
+          mma_commit(&s_full[1]);
+          mma_commit(&k_empty[ks]);
+          ++kcnt;
+        }
+        if (!ok) break;
+        // The last tile's P V products.
+        ok = mbar_wait(&p_full[0], pph[0], kDevTimeoutMma);
+        if (!ok) break;
+        pph[0] ^= 1;
+        const int vs = vcnt % NSV;
+        ok = mbar_wait(&v_full[vs], (vcnt / NSV) & 1, kDevTimeoutMma);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(0, vs, nt > 1);
+        mma_commit(&o_full[0]);
+        ok = mbar_wait(&p_full[1], pph[1], kDevTimeoutMma);
+        if (!ok) break;
+        pph[1] ^= 1;
+        tc_fence_after();
+        issue_pv(1, vs, nt > 1);
+        mma_commit(&v_empty[vs]);
+        ++vcnt;
+        mma_commit(&o_full[1]);
+      }
+      if (issued) {
+        // Every MMA this thread issued has completed before TMEM is released.
+        mma_commit(drain);
+        mbar_wait(drain, 0, kDevTimeoutMma);
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------------ softmax warpgroups
+    const int wg = (warp - 4) / 4;
+    const int wq = warp % 4;
+    const int row = wq * 32 + lane;
+    const uint32_t tl = tbase + ((uint32_t)(wq * 32) << 16);
+    const uint32_t tS = tl + wg * 128;
+    const uint32_t tO = tl + 256 + wg * 128;
+    uint8_t* sQ = smem + S::kQ0 + wg * S::kTile;
+    uint32_t sph = 0, oph = 0;
+    bool ok = true;
+
+    for (int idx = blockIdx.x; idx < p.num_items && ok; idx += gridDim.x) {
+      const Item it = decode_item<MODE>(p, idx);
+      const int nt = it.a_tiles + it.b_tiles;
+      const RowInfo ri = row_info<MODE>(p, it, wg, row);
+      load_q_row<D>(p, it, ri, sQ, row);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&q_full[wg]);
+
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j < nt; ++j) {
+        ok = mbar_wait(&s_full[wg], sph, kDevTimeoutSoftmax);
+        if (!ok) break;
+        sph ^= 1;
+        tc_fence_after();
+        uint32_t sr[kKeys];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+        tmem_ld_wait();
+        const int k0 = tile_key0(it, j);
+        if (k0 + kKeys - 1 > ri.cache_idx) {
+          const int lim = ri.cache_idx - k0;  // keys k0 + c with c > lim are not visible
+#pragma unroll
+          for (int c = 0; c < kKeys; ++c)
+            if (c > lim) sr[c] = __float_as_uint(-INFINITY);
+        }
+        // Row max of the raw scores (scale > 0 commutes with max).
+        float mt = __uint_as_float(sr[0]);
+#pragma unroll
+        for (int c = 1; c < kKeys; ++c) mt = fmaxf(mt, __uint_as_float(sr[c]));
+        const float m_new = fmaxf(m, mt * p.scale_log2);
+        float f = 1.f;
+        const bool rescale = m_new > m + kRescaleThreshold;
+        if (rescale) {
+          f = (l > 0.f) ? ex2_approx(m - m_new) : 1.f;
+          m = m_new;
+        }
+        const float mu = (m == -INFINITY) ? 0.f : m;
+        // P = 2^(s*scale - m), rounded to bf16; l sums the rounded values.
+        uint32_t pk[kKeys / 2];
+        float rs = 0.f;
+#pragma unroll
+        for (int c = 0; c < kKeys / 2; ++c) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * c]), p.scale_log2, -mu));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * c + 1]), p.scale_log2, -mu));
+          pk[c] = pack_bf16x2(p0, p1);
+          const float2 r2 = unpack_bf16x2(pk[c]);
+          rs += r2.x + r2.y;
+        }
+        tmem_st32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+        tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+        l = l * f + rs;
+        if (rescale && f != 1.f) {
+          // O_w holds the products of tiles < j only (its P V for tile j is not
+          // issued before p_full), so it can be scaled in place.
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + c * 32, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+            tmem_st32(tO + c * 32, o);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_full[wg]);
+      }
+      if (!ok) break;
+      ok = mbar_wait(&o_full[wg], oph, kDevTimeoutSoftmax);
+      if (!ok) break;
+      oph ^= 1;
+      tc_fence_after();
+      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+      if (MODE == 0) {
+        bf16* dst = p.out_bf16 + (((size_t)it.bi * p.L + ri.tok) * p.Hq + ri.head) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + c * 32, o);
+          tmem_ld_wait();
+          uint32_t w[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) d4[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+        }
+      } else {
+        const size_t rowoff = (((size_t)it.part * p.B + it.bi) * p.Ntok + ri.tok) * p.Hq + ri.head;
+        float* dst = p.out_f32 + rowoff * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + c * 32, o);
+          tmem_ld_wait();
+          if (ri.valid) {
+            float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              d4[e] = make_float4(__uint_as_float(o[4 * e]) * inv_l, __uint_as_float(o[4 * e + 1]) * inv_l,
+                                  __uint_as_float(o[4 * e + 2]) * inv_l, __uint_as_float(o[4 * e + 3]) * inv_l);
+          }
+        }
+        if (ri.valid) {
+          const float lse = (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+          p.lse_f32[rowoff] = lse;
+        }
+      }
+      tc_fence_before();
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// Pool [num_pages][Hkv][P][d] bf16 as a 4-D tensor (d innermost); box = 64 x 128 x 1 x 1.
+bool make_pool_map(CUtensorMap* map, void* pool, int d, int P, int Hkv, int num_pages) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)P, (cuuint64_t)Hkv, (cuuint64_t)num_pages};
+  const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)P * d * 2, (cuuint64_t)Hkv * P * d * 2};
+  const cuuint32_t box[4] = {64, (cuuint32_t)kKeys, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, pool, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int pow2_at_least(int x) {
+  int v = 1;
+  while (v < x) v <<= 1;
+  return v;
+}
+
+template <int D, int MODE>
+cudaError_t launch_typed(const AttnLaunch& a, const Params& p, const CUtensorMap& mk, const CUtensorMap& mv,
+                         cudaStream_t st) {
+  constexpr int NSK = (D == 128) ? 2 : 4;
+  constexpr int NSV = (D == 128) ? 2 : 4;
+  using S = Smem<D, MODE, NSK, NSV>;
+  auto kern = star_attn_kernel<D, MODE, NSK, NSV>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = std::min(p.num_items, sms);
+  if (grid <= 0) return cudaSuccess;
+  kern<<<grid, kThreads, S::kBytes, st>>>(mk, mv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int attn_num_parts(const AttnLaunch& a) { return a.n * a.chunks_per_block; }
+
+cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t st, const char** why) {
+  Params p;
+  memset(&p, 0, sizeof(p));
+  p.q = reinterpret_cast<const bf16*>(a.q);
+  p.q_pos = a.q_pos;
+  p.out_bf16 = reinterpret_cast<bf16*>(a.out_bf16);
+  p.out_f32 = a.out_f32;
+  p.lse_f32 = a.lse_f32;
+  p.page_table = a.cache.page_table;
+  p.max_pages = a.cache.max_pages;
+  p.num_pages = a.cache.num_pages;
+  p.P = a.cache.P;
+  p.B = a.B;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.G = a.Hq / a.Hkv;
+  p.L = a.L;
+  p.b = a.b;
+  p.n = a.n;
+  p.Ntok = a.Ntok;
+  p.scale_log2 = a.scale_log2;
+  for (int j = 0; j < a.d / 2; ++j) p.inv_freq[j] = a.rope.inv_freq[j];
+  if (a.mode == 0) {
+    p.num_items = a.B * a.Hkv * a.n * (a.b / kRows) * (p.G / 2);
+  } else {
+    p.chunks_per_block = a.chunks_per_block;
+    p.chunk_keys = a.b / a.chunks_per_block;
+    p.tail_tiles = (a.Ntok + kKeys - 1) / kKeys;
+    p.TQ = std::min(pow2_at_least(a.Ntok), kRows);
+    p.HT = kRows / p.TQ;
+    p.NTT = (a.Ntok + p.TQ - 1) / p.TQ;
+    p.NHT = (p.G + p.HT - 1) / p.HT;
+    p.npairs = (p.NTT * p.NHT + 1) / 2;
+    p.num_items = a.n * a.chunks_per_block * a.B * a.Hkv * p.npairs;
+  }
+  CUtensorMap mk, mv;
+  if (!make_pool_map(&mk, a.cache.k_pool, a.d, a.cache.P, a.Hkv, a.cache.num_pages) ||
+      !make_pool_map(&mv, a.cache.v_pool, a.d, a.cache.P, a.Hkv, a.cache.num_pages)) {
+    if (why) *why = "cuTensorMapEncodeTiled failed for the KV pools";
+    return cudaErrorInvalidValue;
+  }
+  if (a.d == 128) {
+    return a.mode == 0 ? launch_typed<128, 0>(a, p, mk, mv, st) : launch_typed<128, 1>(a, p, mk, mv, st);
+  } else {
+    return a.mode == 0 ? launch_typed<64, 0>(a, p, mk, mv, st) : launch_typed<64, 1>(a, p, mk, mv, st);
+  }
+}
+
+cudaError_t read_and_clear_device_error(int* code, cudaStream_t st) {
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return e;
+  e = cudaMemcpyFromSymbol(code, g_device_error, sizeof(int));
+  if (e != cudaSuccess) return e;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+}
+
+}  // namespace star

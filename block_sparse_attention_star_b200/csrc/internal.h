@@ -1,0 +1,82 @@
+// Internal launch interfaces between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace star {
+
+constexpr int kMaxHalfDimHost = 64;
+
+struct RopeTable {
+  double inv_freq[kMaxHalfDimHost];   // theta^(-2j/d), j < d/2
+};
+
+// Paged KV cache view (see star.h: pools are [num_pages][Hkv][P][d] bf16).
+struct CacheView {
+  void* k_pool;
+  void* v_pool;
+  const int32_t* page_table;
+  int max_pages;
+  int num_pages;
+  int P;
+};
+
+// --- rope_append.cu -------------------------------------------------------
+// RoPE(K) at `pos` and copy of V for ntok tokens per sequence, written at cache
+// slots [start, start + ntok).  k/v: [B][ntok][Hkv][d] bf16, pos: [B][ntok].
+cudaError_t launch_rope_append(const void* k, const void* v, const int32_t* pos, int B, int ntok, int start,
+                               int Hkv, int d, const CacheView& c, const RopeTable& rt, cudaStream_t st);
+// Zero cache slots [from, to) of every sequence (K and V).
+cudaError_t launch_zero_slots(int B, int from, int to, int Hkv, int d, const CacheView& c, cudaStream_t st);
+// c' position ids [B][L + (n-1) b] and block map [B][L][3].
+cudaError_t launch_build_positions(const int32_t* pos_ctx, int B, int L, int b, const CacheView& c,
+                                   int32_t* aug_pos, int32_t* block_map, cudaStream_t st);
+
+// --- merge.cu ---------------------------------------------------------------
+// groups x rows outputs; group g merges input parts [g*parts_per_group, (g+1)*parts_per_group).
+// o_in: [parts][rows][d] f32, lse_in: [parts][rows].  Output bf16 or f32 [groups][rows][d].
+cudaError_t launch_lse_merge(int groups, int parts_per_group, int64_t rows, int d, const float* o_in,
+                             const float* lse_in, void* o_out, bool out_bf16, float* lse_out, cudaStream_t st);
+
+// --- attn_sm100.cu ------------------------------------------------------------
+struct AttnLaunch {
+  int mode;               // 0: Phase-1 context attention, 1: Phase-2 query partials
+  int B, Hq, Hkv, d, L, b, n;
+  const void* q;          // [B][Ntok][Hq][d] bf16 (pre-RoPE)
+  const int32_t* q_pos;   // [B][Ntok]
+  int Ntok;
+  CacheView cache;
+  void* out_bf16;         // mode 0: [B][L][Hq][d]
+  float* out_f32;         // mode 1: [parts][B][T][Hq][d]
+  float* lse_f32;         // mode 1: [parts][B][T][Hq]
+  int chunks_per_block;   // mode 1
+  float scale_log2;
+  RopeTable rope;
+};
+int attn_num_parts(const AttnLaunch& a);  // mode 1: n * chunks_per_block
+cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t st, const char** why);
+
+// --- decode.cu ----------------------------------------------------------------
+struct DecodeLaunch {
+  int B, Hq, Hkv, d;
+  const void* q;          // [B][Hq][d] bf16 (pre-RoPE)
+  const int32_t* pos;     // [B] position of the decoded token
+  int n_keys;             // keys [0, n_keys) of every sequence
+  int chunk;              // keys per CTA
+  CacheView cache;
+  float* o_ws;            // [nchunks][B*Hq][d]
+  float* lse_ws;          // [nchunks][B*Hq]
+  float scale_log2;
+  RopeTable rope;
+};
+int decode_num_chunks(int n_keys, int chunk);
+int decode_pick_chunk(int B, int Hkv, int G, int n_keys, int num_sms);
+size_t decode_smem_bytes(int d, int G, int chunk);
+cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t st);
+
+// --- device error word ---------------------------------------------------------
+cudaError_t read_and_clear_device_error(int* code, cudaStream_t st);
+
+}  // namespace star

@@ -1,0 +1,182 @@
+// KV-cache writes of the Star Attention hot path (HBM-bound, no tensor cores).
+//
+// * rope_append: K rotated by RoPE at the token's position id and V copied,
+//   both bf16, into the paged cache.  Phase 1 writes only the L context tokens
+//   -- never the (n-1)*b anchor copies of c' ("Star Attention 完全拆解(一)",
+//   "局部注意力与 KV 丢弃": the anchor's KV is discarded, and it equals block 1's
+//   since the anchor keeps block 1's positions).  Phase 2 and decode append the
+//   query / generated tokens at the tail of the last block ("仓库里的真实实现":
+//   only the last host extends its cache).
+// * zero_slots: clears cache slots past the context so that tiles which run over
+//   the valid tail hold zeros, not stale values (masked keys get P = 0, and
+//   0 * V must stay 0).
+// * build_positions: the integer position ids of c' and the token -> (block,
+//   page, slot) map ("被增广的上下文").
+//
+// Layout: pools are [num_pages][Hkv][P][d] bf16; logical page t / P of sequence
+// bi is physical page page_table[bi * max_pages + t / P]; slot t % P.
+// Each thread moves 16 bytes: for K, eight rotation pairs (x_j, x_{j+d/2}).
+#include "common.cuh"
+#include "internal.h"
+
+namespace star {
+namespace {
+
+struct RopeParams {
+  double inv_freq[kMaxHalfDim];
+};
+
+template <int D>
+__global__ void __launch_bounds__(256) rope_append_kernel(const bf16* __restrict__ k, const bf16* __restrict__ v,
+                                                          const int32_t* __restrict__ pos, int B, int ntok, int start,
+                                                          int Hkv, bf16* __restrict__ kpool, bf16* __restrict__ vpool,
+                                                          const int32_t* __restrict__ page_table, int max_pages,
+                                                          int num_pages, int P, const __grid_constant__ RopeParams rp) {
+  constexpr int CH = D / 16;  // threads per (token, head) row: 8 pairs each
+  const long long total = (long long)B * ntok * Hkv * CH;
+  for (long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x; gid < total;
+       gid += (long long)gridDim.x * blockDim.x) {
+    const int c = (int)(gid % CH);
+    long long r = gid / CH;
+    const int h = (int)(r % Hkv);
+    r /= Hkv;
+    const int t = (int)(r % ntok);
+    const int bi = (int)(r / ntok);
+    const size_t src = (((size_t)bi * ntok + t) * Hkv + h) * D;
+    const int slot_abs = start + t;
+    const int page = page_table[(size_t)bi * max_pages + slot_abs / P];
+    if (page < 0 || page >= num_pages) {
+      record_error(kDevBadPage);
+      continue;
+    }
+    const size_t dst = (((size_t)page * Hkv + h) * P + (slot_abs % P)) * D;
+    const int p_t = pos[(size_t)bi * ntok + t];
+
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(k + src + 8 * c));
+    const uint4 bq = __ldg(reinterpret_cast<const uint4*>(k + src + D / 2 + 8 * c));
+    const uint32_t* aw = reinterpret_cast<const uint32_t*>(&a);
+    const uint32_t* bw = reinterpret_cast<const uint32_t*>(&bq);
+    uint32_t lo[4], hi[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 x1 = unpack_bf16x2(aw[e]);
+      const float2 x2 = unpack_bf16x2(bw[e]);
+      float c0, s0, c1, s1;
+      rope_sincos(p_t, rp.inv_freq[8 * c + 2 * e], c0, s0);
+      rope_sincos(p_t, rp.inv_freq[8 * c + 2 * e + 1], c1, s1);
+      lo[e] = pack_bf16x2(x1.x * c0 - x2.x * s0, x1.y * c1 - x2.y * s1);
+      hi[e] = pack_bf16x2(x2.x * c0 + x1.x * s0, x2.y * c1 + x1.y * s1);
+    }
+    *reinterpret_cast<uint4*>(kpool + dst + 8 * c) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    *reinterpret_cast<uint4*>(kpool + dst + D / 2 + 8 * c) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    // V: the same thread copies the two 16-byte chunks at the same offsets.
+    *reinterpret_cast<uint4*>(vpool + dst + 8 * c) = __ldg(reinterpret_cast<const uint4*>(v + src + 8 * c));
+    *reinterpret_cast<uint4*>(vpool + dst + D / 2 + 8 * c) =
+        __ldg(reinterpret_cast<const uint4*>(v + src + D / 2 + 8 * c));
+  }
+}
+
+__global__ void zero_slots_kernel(int B, int from, int to, int Hkv, int d, bf16* kpool, bf16* vpool,
+                                  const int32_t* page_table, int max_pages, int num_pages, int P) {
+  const int CH = d / 8;
+  const long long span = to - from;
+  const long long total = (long long)B * span * Hkv * CH;
+  for (long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x; gid < total;
+       gid += (long long)gridDim.x * blockDim.x) {
+    const int c = (int)(gid % CH);
+    long long r = gid / CH;
+    const int h = (int)(r % Hkv);
+    r /= Hkv;
+    const int s = from + (int)(r % span);
+    const int bi = (int)(r / span);
+    const int page = page_table[(size_t)bi * max_pages + s / P];
+    if (page < 0 || page >= num_pages) {
+      record_error(kDevBadPage);
+      continue;
+    }
+    const size_t off = (((size_t)page * Hkv + h) * P + (s % P)) * d + 8 * c;
+    *reinterpret_cast<uint4*>(kpool + off) = make_uint4(0, 0, 0, 0);
+    *reinterpret_cast<uint4*>(vpool + off) = make_uint4(0, 0, 0, 0);
+  }
+}
+
+// Augmented row a of sequence bi: block 0 holds rows [0, b); block i >= 1 holds
+// rows [b + 2b(i-1), b + 2b i): b anchor rows (ids of tokens 0..b-1) then its own.
+__global__ void build_positions_kernel(const int32_t* pos_ctx, int B, int L, int b, const int32_t* page_table,
+                                       int max_pages, int P, int32_t* aug_pos, int32_t* block_map) {
+  const int n = L / b;
+  const long long aug_len = (long long)L + (long long)(n - 1) * b;
+  const long long total = (long long)B * aug_len;
+  for (long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x; gid < total;
+       gid += (long long)gridDim.x * blockDim.x) {
+    const int bi = (int)(gid / aug_len);
+    const long long a = gid % aug_len;
+    long long tok;
+    if (a < b) {
+      tok = a;
+    } else {
+      const long long i = 1 + (a - b) / (2LL * b);
+      const long long off = (a - b) % (2LL * b);
+      tok = off < b ? off : i * b + (off - b);
+    }
+    aug_pos[gid] = pos_ctx[(size_t)bi * L + tok];
+  }
+  const long long total_map = (long long)B * L;
+  for (long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x; gid < total_map;
+       gid += (long long)gridDim.x * blockDim.x) {
+    const int bi = (int)(gid / L);
+    const int t = (int)(gid % L);
+    block_map[3 * gid + 0] = t / b;
+    block_map[3 * gid + 1] = page_table[(size_t)bi * max_pages + t / P];
+    block_map[3 * gid + 2] = t % P;
+  }
+}
+
+int grid_for(long long work, int threads) {
+  long long g = (work + threads - 1) / threads;
+  if (g < 1) g = 1;
+  if (g > 148LL * 64) g = 148LL * 64;
+  return (int)g;
+}
+
+}  // namespace
+
+cudaError_t launch_rope_append(const void* k, const void* v, const int32_t* pos, int B, int ntok, int start, int Hkv,
+                               int d, const CacheView& c, const RopeTable& rt, cudaStream_t st) {
+  if (ntok <= 0 || B <= 0) return cudaSuccess;
+  RopeParams rp;
+  for (int j = 0; j < d / 2; ++j) rp.inv_freq[j] = rt.inv_freq[j];
+  const long long work = (long long)B * ntok * Hkv * (d / 16);
+  const int grid = grid_for(work, 256);
+  if (d == 128) {
+    rope_append_kernel<128><<<grid, 256, 0, st>>>(
+        reinterpret_cast<const bf16*>(k), reinterpret_cast<const bf16*>(v), pos, B, ntok, start, Hkv,
+        reinterpret_cast<bf16*>(c.k_pool), reinterpret_cast<bf16*>(c.v_pool), c.page_table, c.max_pages,
+        c.num_pages, c.P, rp);
+  } else {
+    rope_append_kernel<64><<<grid, 256, 0, st>>>(
+        reinterpret_cast<const bf16*>(k), reinterpret_cast<const bf16*>(v), pos, B, ntok, start, Hkv,
+        reinterpret_cast<bf16*>(c.k_pool), reinterpret_cast<bf16*>(c.v_pool), c.page_table, c.max_pages,
+        c.num_pages, c.P, rp);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_zero_slots(int B, int from, int to, int Hkv, int d, const CacheView& c, cudaStream_t st) {
+  if (to <= from) return cudaSuccess;
+  const long long work = (long long)B * (to - from) * Hkv * (d / 8);
+  zero_slots_kernel<<<grid_for(work, 256), 256, 0, st>>>(B, from, to, Hkv, d, reinterpret_cast<bf16*>(c.k_pool),
+                                                          reinterpret_cast<bf16*>(c.v_pool), c.page_table,
+                                                          c.max_pages, c.num_pages, c.P);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_build_positions(const int32_t* pos_ctx, int B, int L, int b, const CacheView& c, int32_t* aug_pos,
+                                   int32_t* block_map, cudaStream_t st) {
+  const long long work = (long long)B * (L + (long long)(L / b - 1) * b);
+  build_positions_kernel<<<grid_for(work, 256), 256, 0, st>>>(pos_ctx, B, L, b, c.page_table, c.max_pages, c.P,
+                                                               aug_pos, block_map);
+  return cudaGetLastError();
+}
+
+}  // namespace star

@@ -1,0 +1,190 @@
+/*
+ * star.h -- C ABI of the Star Attention hot path on NVIDIA B200 (sm_100a).
+ *
+ * Star Attention ("Star Attention: Efficient LLM Inference over Long
+ * Sequences"; walk-through in "Star Attention 完全拆解(一):锚点块、分块上下文编码
+ * 与两阶段全局注意力") is a two-phase block-sparse approximation of attention:
+ *
+ *   Phase 1 (context encoding): the context c = [c_1 .. c_n] of L = n*b tokens is
+ *     split into blocks of b tokens; every block after the first is prefixed by
+ *     the anchor block c_1, which keeps its own position ids, and runs causal
+ *     attention locally; the anchor's KV is discarded and only c_i's is cached.
+ *   Phase 2 (query and generation): query and generated tokens attend to every
+ *     cached block; each block yields a local (output, log-sum-exp) pair and the
+ *     pairs are merged exactly into global attention.
+ *
+ * Conventions for every call below
+ *   - One attention layer.  Q, K, V are that layer's projections (pre-RoPE).
+ *   - Tensor pointers are DEVICE pointers owned by the caller, contiguous,
+ *     16-byte aligned; bf16 means IEEE bfloat16.  Layout is [B, tokens, heads, d]
+ *     ("bshd") unless stated.  Position ids are int32.
+ *   - The library allocates no device memory.  Scratch space is passed in as
+ *     `ws` of at least star_workspace_size() bytes.
+ *   - Every call is asynchronous on the caller's CUDA stream `stream` (a
+ *     cudaStream_t; NULL = legacy default stream) and never synchronises, except
+ *     star_device_status().
+ *   - Return value: STAR_OK (0) or a negative STAR_ERR_* code; star_last_error()
+ *     then describes the failure (thread-local).  Arguments are validated on the
+ *     host before anything is launched; a failing call launches nothing.
+ *   - RoPE: rotate-half pairing (x_j, x_{j+d/2}), inv_freq_j = theta^(-2j/d),
+ *     angle pos * inv_freq_j formed in float64; rotated Q and K are rounded to
+ *     bf16.  Softmax scale 1/sqrt(d).  GQA: query head h uses KV head h / (Hq/Hkv).
+ *   - LSE values are natural logarithms: log sum_k exp(q.k / sqrt(d)).
+ */
+#ifndef STAR_H_
+#define STAR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* star_stream_t; /* == cudaStream_t */
+
+enum {
+  STAR_OK = 0,
+  STAR_ERR_INVALID_ARG = -1,      /* null pointer, negative size, inconsistent shape */
+  STAR_ERR_UNSUPPORTED_SHAPE = -2,/* valid but not supported: d not in {64,128}, odd Hq/Hkv, L != n*b, ... */
+  STAR_ERR_ALIGNMENT = -3,        /* a pointer is not 16-byte aligned */
+  STAR_ERR_CAPACITY = -4,         /* page table / pool / workspace too small */
+  STAR_ERR_CUDA = -5,             /* a CUDA runtime or driver call failed */
+  STAR_ERR_TIMEOUT = -6           /* a kernel gave up a bounded wait (see star_device_status) */
+};
+
+/* Workspace query selectors. */
+enum { STAR_OP_PHASE1 = 1, STAR_OP_PHASE2 = 2, STAR_OP_DECODE = 3 };
+
+/* Problem shape ("问题定义与记号": context c of n blocks of b tokens, query q). */
+typedef struct star_shape {
+  int32_t B;           /* independent sequences */
+  int32_t Hq;          /* query heads; Hq / Hkv must be even (2, 4, 8) */
+  int32_t Hkv;         /* key/value heads */
+  int32_t d;           /* head dim: 64 or 128 */
+  int32_t L;           /* context tokens, L = n * b */
+  int32_t b;           /* block size (anchor size = b); multiple of 128 and of page_tokens */
+  int32_t n;           /* number of blocks */
+  int32_t T_max;       /* tail capacity after the context: query + generated tokens */
+  int32_t page_tokens; /* P: tokens per cache page; multiple of 128 */
+  double rope_theta;   /* RoPE base, e.g. 500000 */
+} star_shape;
+
+/* Paged KV cache ("局部注意力与 KV 丢弃": only non-anchor KV is kept).
+ * k_pool, v_pool: bf16 [num_pages][Hkv][page_tokens][d]; one (page, head) run is
+ * page_tokens*d*2 contiguous bytes.  Token t of sequence s lives in physical page
+ * page_table[s*max_pages + t/page_tokens], slot t % page_tokens; K is stored
+ * after RoPE, V as given.  page_table is a DEVICE int32 array [B][max_pages]
+ * that the caller fills (star_page_table_fill gives the block-contiguous one:
+ * block i of a sequence occupies consecutive physical pages).  It must cover
+ * tokens [0, L + round_up(T_max, 128)). */
+typedef struct star_cache {
+  void* k_pool;
+  void* v_pool;
+  const int32_t* page_table;
+  int32_t max_pages;   /* logical pages per sequence */
+  int32_t num_pages;   /* physical pages in each pool */
+} star_cache;
+
+/* Library version string (static storage). */
+const char* star_version(void);
+
+/* Message of the last failing call on this thread ("" if none). Static storage,
+ * valid until the next failing call on the same thread. */
+const char* star_last_error(void);
+
+/* Logical pages one sequence needs: ceil((L + round_up(T_max,128)) / page_tokens). */
+int star_pages_needed(const star_shape* shape, int32_t* max_pages_out);
+
+/* HOST helper: fill a host int32 array [B][max_pages] with the block-contiguous
+ * assignment page_table[s][j] = first_page + s*max_pages + j. */
+int star_page_table_fill(const star_shape* shape, int32_t* page_table_host, int32_t max_pages, int32_t first_page);
+
+/* Bytes of scratch the given operation needs (op = STAR_OP_*; for STAR_OP_PHASE2
+ * T is the number of query tokens of the call, ignored otherwise). */
+int star_workspace_size(const star_shape* shape, int op, int32_t T, size_t* bytes_out);
+
+/* Integer structure of c' ("被增广的上下文"), for checking only.
+ * pos_ctx:   device int32 [B][L], position id of each context token (normally t).
+ * aug_pos:   device int32 [B][L + (n-1)*b], position ids of c' = [c_1, (c_1 c_2), ...,
+ *            (c_1 c_n)]: block 1 then, per block i>1, b anchor ids then c_i's ids.
+ * block_map: device int32 [B][L][3]: (block t/b, physical page, slot t % page_tokens).
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE (L != n*b), CAPACITY, CUDA. */
+int star_build_positions(const star_shape* shape, const star_cache* cache, const int32_t* pos_ctx,
+                         int32_t* aug_pos, int32_t* block_map, star_stream_t stream);
+
+/* Append tokens to the cache ("仓库里的真实实现": the last block's owner appends the
+ * query and generated tokens' KV; "局部注意力与 KV 丢弃" for the context).
+ * k, v: bf16 [B][ntok][Hkv][d]; pos: device int32 [B][ntok] (RoPE positions of K).
+ * Writes RoPE(K) and V into cache slots [start, start + ntok) of every sequence.
+ * Errors: INVALID_ARG, ALIGNMENT, CAPACITY (start + ntok beyond the page table), CUDA. */
+int star_kv_append(const star_shape* shape, const star_cache* cache, const void* k, const void* v,
+                   const int32_t* pos, int32_t start, int32_t ntok, star_stream_t stream);
+
+/* Phase 1: anchor-augmented blockwise-local causal attention plus the KV cache
+ * ("Phase 1: 被增广的上下文", "局部注意力与 KV 丢弃", "复杂度分析").
+ * q: bf16 [B][L][Hq][d]; k, v: bf16 [B][L][Hkv][d]; pos_ctx: device int32 [B][L].
+ * Writes out: bf16 [B][L][Hq][d], where row t of block i attends to the anchor
+ * keys [0, b) (for i > 1) and to its own block's keys up to t, each key roped at
+ * its own position id.  Writes RoPE(K), V of the L context tokens into cache
+ * slots [0, L) (the anchor copies are never written) and zeroes slots
+ * [L, L + round_up(T_max,128)).
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, ALIGNMENT, CAPACITY, CUDA. */
+int star_phase1_encode(const star_shape* shape, const star_cache* cache, const void* q, const void* k,
+                       const void* v, const int32_t* pos_ctx, void* out, void* ws, size_t ws_bytes,
+                       star_stream_t stream);
+
+/* Phase 2 per-block partials ("Phase 2: 局部注意力与本地统计量": A_h and s_h per host).
+ * q: bf16 [B][T][Hq][d]; k, v: bf16 [B][T][Hkv][d] or both NULL (already appended);
+ * q_pos: device int32 [B][T], RoPE positions (normally L + t).
+ * If k, v are given they are appended first at cache slots [L, L+T) (tail of the
+ * last block).  Query token t (cache index L + t) sees all keys of blocks 1..n-1
+ * and, in block n, its b context keys plus tail keys L..L+t.
+ * o_part: f32 [n][B][T][Hq][d], normalised local outputs A_i;
+ * lse_part: f32 [n][B][T][Hq], log s_i.  T <= T_max.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, ALIGNMENT, CAPACITY, CUDA. */
+int star_phase2_partial(const star_shape* shape, const star_cache* cache, const void* q, const void* k,
+                        const void* v, const int32_t* q_pos, int32_t T, float* o_part, float* lse_part, void* ws,
+                        size_t ws_bytes, star_stream_t stream);
+
+/* Exact merge of partials ("组装全局结果"; log-sum-exp form of "数值稳定性").
+ * o_part: f32 [n_parts][rows][d]; lse_part: f32 [n_parts][rows].
+ * out: bf16 [rows][d] = sum_i exp(LSE_i - LSE) O_i; lse_out: f32 [rows] =
+ * log sum_i exp(LSE_i) (may be NULL).  Partials with non-finite LSE are skipped;
+ * a row with none gives O = 0, LSE = -inf.  With the layouts of
+ * star_phase2_partial, rows = B*T*Hq.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE (d), ALIGNMENT, CUDA. */
+int star_lse_merge(int32_t n_parts, int64_t rows, int32_t d, const float* o_part, const float* lse_part, void* out,
+                   float* lse_out, star_stream_t stream);
+
+/* One generated token per sequence ("Star Attention: Efficient LLM Inference over
+ * Long Sequences", abstract: response tokens attend to all prior cached tokens).
+ * q: bf16 [B][1][Hq][d]; k, v: bf16 [B][1][Hkv][d]; pos: device int32 [B].
+ * Appends RoPE(k), v at cache slot cur_len, then attends over slots [0, cur_len]
+ * (the whole cache including the new token), split into chunks whose (O, LSE)
+ * partials are merged exactly.  out: bf16 [B][1][Hq][d]; lse_out: f32 [B][Hq]
+ * (may be NULL).  cur_len < L + T_max.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, ALIGNMENT, CAPACITY, CUDA. */
+int star_decode_step(const star_shape* shape, const star_cache* cache, const void* q, const void* k, const void* v,
+                     const int32_t* pos, int32_t cur_len, void* out, float* lse_out, void* ws, size_t ws_bytes,
+                     star_stream_t stream);
+
+/* Tracing: when both are non-NULL (cudaEvent_t handles created by the caller),
+ * every later call on this thread records `start_event` on its stream right
+ * before launching its main kernel and `stop_event` right after it (Phase 1 and
+ * Phase 2: the tensor-core attention kernel; decode: the split-KV kernel), so the
+ * caller can time that kernel with cudaEventElapsedTime.  NULL, NULL turns it off.
+ * Errors: INVALID_ARG if exactly one is NULL. */
+int star_set_trace_events(void* start_event, void* stop_event);
+
+/* Synchronises `stream`, then reads and clears the device error word that the
+ * kernels set when a bounded wait runs out or a page-table entry is out of range.
+ * *status_out receives the raw code (0 = none).  Returns STAR_ERR_TIMEOUT if a wait
+ * ran out, STAR_ERR_CAPACITY for a bad page, STAR_ERR_CUDA if the stream failed. */
+int star_device_status(star_stream_t stream, int32_t* status_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STAR_H_ */

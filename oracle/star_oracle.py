@@ -245,17 +245,19 @@ def phase1_rows(rows, q_rows: np.ndarray, k: np.ndarray, v: np.ndarray, pos_ctx,
             cache[i] = rope_bf16(k[tok], pos_ctx[tok], theta)
         return cache[i]
 
-    for r_i, t in enumerate(rows):
-        i = int(t) // b
-        own = np.arange(i * b, int(t) + 1)
-        keys = roped_block(i)[: len(own)]
-        vals = np.asarray(v[own], dtype=np.float64)
+    for i in np.unique(rows // b):
+        sel = np.nonzero(rows // b == i)[0]
+        own = np.arange(i * b, (i + 1) * b)
+        keys, vals, key_idx = roped_block(i), np.asarray(v[own], dtype=np.float64), own
         if i > 0:
             keys = np.concatenate([roped_block(0), keys])
             vals = np.concatenate([np.asarray(v[:b], dtype=np.float64), vals])
-        qr = rope_bf16(q_rows[r_i: r_i + 1], pos_ctx[[t]], theta)
-        O, _ = attend(qr, keys, vals)
-        out[r_i] = O[0]
+            key_idx = np.concatenate([np.arange(b), own])
+        # augmented row of token t sees the anchor (all of it) and its own block up to t
+        vis = key_idx[None, :] <= rows[sel][:, None]
+        qr = rope_bf16(q_rows[sel], pos_ctx[rows[sel]], theta)
+        O, _ = attend(qr, keys, vals, vis)
+        out[sel] = O
     return out
 
 

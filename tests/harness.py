@@ -1,0 +1,109 @@
+"""Shared helpers for the parity tests and the smoke check.
+
+Runs the whole hot path of one workload through the C-ABI binding (GPU) and
+through the oracle (CPU) on the same seeded inputs, and compares the results
+with the stated tolerances.
+"""
+
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+import torch
+
+import block_sparse_attention_star_b200 as star
+from synth import Workload, make_inputs
+
+# Floating-point tolerances: bf16 inputs, fp32 accumulation.
+MAX_ABS = 1.5e-2
+MEAN_ABS = 2e-3
+LSE_ABS = 1e-3
+
+
+def shape_of(wl: Workload) -> star.StarShape:
+    return star.StarShape.make(B=wl.B, Hq=wl.Hq, Hkv=wl.Hkv, d=wl.d, L=wl.L, b=wl.b, T_max=wl.T_max,
+                               page_tokens=wl.page_tokens, rope_theta=wl.theta)
+
+
+def to64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def run_gpu(wl: Workload, inp: dict, page_table: torch.Tensor | None = None, num_pages: int | None = None,
+            phases=("phase1", "phase2", "decode")) -> dict:
+    """All steps of the hot path on the current CUDA device; returns device tensors."""
+    dev = inp["q_ctx"].device
+    shape = shape_of(wl)
+    cache = star.PagedKVCache(shape, device=dev, page_table=page_table, num_pages=num_pages)
+    res = {"cache": cache, "shape": shape}
+    if "phase1" in phases:
+        out = torch.empty_like(inp["q_ctx"])
+        star.star_phase1_encode(shape, cache, inp["q_ctx"], inp["k_ctx"], inp["v_ctx"], inp["pos_ctx"], out)
+        res["o_ctx"] = out
+    if "phase2" in phases:
+        T = wl.T
+        o_part, lse_part = star.alloc_partials(shape, T, dev)
+        ws = star.workspace(shape, star.STAR_OP_PHASE2, T, dev)
+        star.star_phase2_partial(shape, cache, inp["q_query"], inp["k_query"], inp["v_query"], inp["pos_query"], T,
+                                 o_part, lse_part, ws)
+        o_q = torch.empty((wl.B, T, wl.Hq, wl.d), dtype=torch.bfloat16, device=dev)
+        lse_q = torch.empty((wl.B, T, wl.Hq), dtype=torch.float32, device=dev)
+        star.star_lse_merge(shape.n, wl.B * T * wl.Hq, wl.d, o_part, lse_part, o_q, lse_q)
+        res.update(o_part=o_part, lse_part=lse_part, o_query=o_q, lse_query=lse_q)
+    if "decode" in phases:
+        wsd = star.workspace(shape, star.STAR_OP_DECODE, 0, dev)
+        o_dec = torch.empty((wl.S, wl.B, 1, wl.Hq, wl.d), dtype=torch.bfloat16, device=dev)
+        lse_dec = torch.empty((wl.S, wl.B, wl.Hq), dtype=torch.float32, device=dev)
+        for s in range(wl.S):
+            star.star_decode_step(shape, cache, inp["q_dec"][s], inp["k_dec"][s], inp["v_dec"][s], inp["pos_dec"][s],
+                                  wl.L + wl.T + s, o_dec[s], lse_dec[s], wsd)
+        res.update(o_dec=o_dec, lse_dec=lse_dec)
+    torch.cuda.synchronize()
+    res["status"] = star.star_device_status()
+    return res
+
+
+def oracle_inputs(inp: dict) -> dict:
+    return {k: (to64(v) if v.dtype == torch.bfloat16 else v.cpu().numpy().astype(np.int64)) for k, v in inp.items()}
+
+
+@dataclasses.dataclass
+class Err:
+    max_abs: float
+    mean_abs: float
+
+    def ok(self, max_abs=MAX_ABS, mean_abs=MEAN_ABS) -> bool:
+        return self.max_abs <= max_abs and self.mean_abs <= mean_abs
+
+
+def err(gpu, ref) -> Err:
+    g = to64(gpu) if isinstance(gpu, torch.Tensor) else np.asarray(gpu, dtype=np.float64)
+    r = np.asarray(ref, dtype=np.float64)
+    assert g.shape == r.shape, (g.shape, r.shape)
+    d = np.abs(g - r)
+    return Err(float(d.max()) if d.size else 0.0, float(d.mean()) if d.size else 0.0)
+
+
+def assert_out(gpu, ref, what: str):
+    e = err(gpu, ref)
+    assert e.ok(), f"{what}: max abs {e.max_abs:.3e} (<= {MAX_ABS}), mean abs {e.mean_abs:.3e} (<= {MEAN_ABS})"
+    return e
+
+
+def assert_lse(gpu, ref, what: str):
+    e = err(gpu, ref)
+    assert e.max_abs <= LSE_ABS, f"{what}: LSE max abs {e.max_abs:.3e} (<= {LSE_ABS})"
+    return e
+
+
+def sample_rows(wl: Workload, per_block: int, seed: int = 0) -> np.ndarray:
+    """Context rows checked at large sizes: {0, 127, 128, b-1} of each block plus seeded random rows."""
+    rng = np.random.default_rng(seed)
+    rows = []
+    for i in range(wl.n):
+        base = i * wl.b
+        fixed = [0, 127, 128, wl.b - 1]
+        rnd = rng.choice(wl.b, size=min(per_block, wl.b), replace=False)
+        rows.extend(base + np.unique(np.concatenate([fixed, rnd])))
+    return np.array(sorted(set(int(r) for r in rows)))

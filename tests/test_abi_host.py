@@ -1,0 +1,75 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every symbol the header declares, and validates shapes and capacities."""
+
+import ctypes
+
+import pytest
+
+import block_sparse_attention_star_b200 as star
+from synth import CONFIGS
+
+
+def test_library_exports_every_header_symbol():
+    lib = star.lib()
+    syms = star.header_symbols()
+    assert len(syms) >= 12
+    for s in syms:
+        assert hasattr(lib, s), s
+    assert star.star_version().startswith("star-b200")
+
+
+def _shape(**kw):
+    base = dict(B=1, Hq=32, Hkv=8, d=128, L=131072, b=32768, T_max=128)
+    base.update(kw)
+    return star.StarShape.make(**base)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(L=131000), star.STAR_ERR_UNSUPPORTED_SHAPE),          # ragged last block
+    (dict(Hq=24, Hkv=8), star.STAR_ERR_UNSUPPORTED_SHAPE),      # group of 3
+    (dict(Hq=30, Hkv=8), star.STAR_ERR_INVALID_ARG),            # not a multiple
+    (dict(d=96), star.STAR_ERR_UNSUPPORTED_SHAPE),
+    (dict(b=32704, L=32704 * 4), star.STAR_ERR_UNSUPPORTED_SHAPE),  # b not a multiple of 128
+    (dict(B=0), star.STAR_ERR_INVALID_ARG),
+    (dict(rope_theta=-1.0), star.STAR_ERR_INVALID_ARG),
+])
+def test_shape_validation(kw, code):
+    with pytest.raises(star.StarError) as e:
+        star.star_pages_needed(_shape(**kw))
+    assert e.value.code == code
+    assert star.lib().star_last_error().decode()
+
+
+def test_pages_and_page_table():
+    sh = _shape()
+    need = star.star_pages_needed(sh)
+    assert need == (131072 + 128 + 255) // 256
+    tab = star.star_page_table_fill(sh, need, first_page=5)
+    assert tab.shape == (1, need) and tab[0, 0] == 5 and tab[0, -1] == 5 + need - 1
+    with pytest.raises(star.StarError) as e:
+        star.star_page_table_fill(sh, need - 1)
+    assert e.value.code == star.STAR_ERR_CAPACITY
+
+
+def test_workspace_sizes_for_every_workload():
+    for wl in CONFIGS.values():
+        sh = star.StarShape.make(B=wl.B, Hq=wl.Hq, Hkv=wl.Hkv, d=wl.d, L=wl.L, b=wl.b, T_max=wl.T_max)
+        assert star.star_workspace_size(sh, star.STAR_OP_PHASE1) == 0
+        ws2 = star.star_workspace_size(sh, star.STAR_OP_PHASE2, wl.T)
+        wsd = star.star_workspace_size(sh, star.STAR_OP_DECODE)
+        assert ws2 % 256 == 0 and wsd % 256 == 0 and wsd > 0
+        with pytest.raises(star.StarError):
+            star.star_workspace_size(sh, star.STAR_OP_PHASE2, wl.T_max + 1)
+
+
+def test_null_arguments_rejected_before_any_launch():
+    lib = star.lib()
+    sh = _shape()
+    rc = lib.star_phase1_encode(ctypes.byref(sh), None, None, None, None, None, None, None, 0, None)
+    assert rc == star.STAR_ERR_INVALID_ARG
+    rc = lib.star_lse_merge(0, 10, 128, None, None, None, None, None)
+    assert rc == star.STAR_ERR_INVALID_ARG
+    rc = lib.star_lse_merge(2, 10, 96, ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.c_void_p(16), None, None)
+    assert rc == star.STAR_ERR_UNSUPPORTED_SHAPE
+    rc = lib.star_set_trace_events(ctypes.c_void_p(16), None)
+    assert rc == star.STAR_ERR_INVALID_ARG
