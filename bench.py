@@ -172,7 +172,44 @@ def _ev():
     return torch.cuda.Event(enable_timing=True)
 
 
+class RawEvent:
+    """A cudaEvent_t created through the CUDA runtime that torch loaded.
+
+    The library records these itself (star_set_trace_events), which torch's Event
+    wrapper does not track, so creation and elapsed time go through the runtime.
+    """
+    _rt = None
+
+    @classmethod
+    def rt(cls):
+        if cls._rt is None:
+            import ctypes
+            torch.cuda.init()
+            cls._rt = ctypes.CDLL("libcudart.so.12")
+        return cls._rt
+
+    def __init__(self):
+        import ctypes
+        h = ctypes.c_void_p()
+        if self.rt().cudaEventCreate(ctypes.byref(h)) != 0:
+            raise RuntimeError("cudaEventCreate failed")
+        self.cuda_event = h.value
+
+    def elapsed_time(self, other) -> float:
+        import ctypes
+        ms = ctypes.c_float()
+        rc = self.rt().cudaEventElapsedTime(ctypes.byref(ms), ctypes.c_void_p(self.cuda_event),
+                                            ctypes.c_void_p(other.cuda_event))
+        if rc != 0:
+            raise RuntimeError(f"cudaEventElapsedTime failed ({rc})")
+        return ms.value
+
+
 def _pair():
+    return (RawEvent(), RawEvent())
+
+
+def _tpair():
     return (_ev(), _ev())
 
 
@@ -194,7 +231,7 @@ def run_star(args, rank, world, local_rank):
 
     K = args.steps
     evs = [{"p1": _pair(), "p2": _pair(), "dec": [_pair() for _ in range(wl.S)],
-            "dec_call": [_pair() for _ in range(wl.S)]} for _ in range(K)]
+            "dec_call": [_tpair() for _ in range(wl.S)]} for _ in range(K)]
     t0, t1 = _ev(), _ev()
     if world > 1:
         dist.barrier()

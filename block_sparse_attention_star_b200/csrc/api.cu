@@ -80,8 +80,8 @@ int64_t pages_needed(const star_shape* s) {
 int check_cache(const star_shape* s, const star_cache* c) {
   if (!c) return fail(STAR_ERR_INVALID_ARG, "cache is NULL");
   if (!c->k_pool || !c->v_pool || !c->page_table) return fail(STAR_ERR_INVALID_ARG, "cache pointers must be non-NULL");
-  if (!aligned16(c->k_pool) || !aligned16(c->v_pool) || !aligned16(c->page_table))
-    return fail(STAR_ERR_ALIGNMENT, "cache pointers must be 16-byte aligned");
+  if (!aligned16(c->k_pool) || !aligned16(c->v_pool) || (reinterpret_cast<uintptr_t>(c->page_table) & 3u))
+    return fail(STAR_ERR_ALIGNMENT, "cache pools must be 16-byte aligned, the page table 4-byte aligned");
   if (c->max_pages < pages_needed(s))
     return fail(STAR_ERR_CAPACITY, "page table has %d pages per sequence, %lld needed", c->max_pages,
                 (long long)pages_needed(s));
@@ -108,6 +108,14 @@ star::RopeTable rope_table(const star_shape* s) {
 }
 
 float scale_log2(const star_shape* s) { return (float)(1.4426950408889634 / std::sqrt((double)s->d)); }
+
+// Position ids and LSE values are accessed one element at a time: 4-byte alignment.
+#define STAR_REQUIRE_PTR4(p, name)                                                   \
+  do {                                                                               \
+    if (!(p)) return fail(STAR_ERR_INVALID_ARG, "%s is NULL", name);                 \
+    if (reinterpret_cast<uintptr_t>(p) & 3u)                                         \
+      return fail(STAR_ERR_ALIGNMENT, "%s is not 4-byte aligned", name);             \
+  } while (0)
 
 #define STAR_REQUIRE_PTR(p, name)                                                    \
   do {                                                                               \
@@ -200,9 +208,9 @@ int star_build_positions(const star_shape* shape, const star_cache* cache, const
   int rc = check_shape(shape);
   if (!rc) rc = check_cache(shape, cache);
   if (rc) return rc;
-  STAR_REQUIRE_PTR(pos_ctx, "pos_ctx");
-  STAR_REQUIRE_PTR(aug_pos, "aug_pos");
-  STAR_REQUIRE_PTR(block_map, "block_map");
+  STAR_REQUIRE_PTR4(pos_ctx, "pos_ctx");
+  STAR_REQUIRE_PTR4(aug_pos, "aug_pos");
+  STAR_REQUIRE_PTR4(block_map, "block_map");
   cudaError_t e = star::launch_build_positions(pos_ctx, shape->B, shape->L, shape->b, view(shape, cache), aug_pos,
                                                block_map, (cudaStream_t)stream);
   return e == cudaSuccess ? STAR_OK : cuda_fail(e, "build_positions launch");
@@ -215,7 +223,7 @@ int star_kv_append(const star_shape* shape, const star_cache* cache, const void*
   if (rc) return rc;
   STAR_REQUIRE_PTR(k, "k");
   STAR_REQUIRE_PTR(v, "v");
-  STAR_REQUIRE_PTR(pos, "pos");
+  STAR_REQUIRE_PTR4(pos, "pos");
   if (start < 0 || ntok < 0) return fail(STAR_ERR_INVALID_ARG, "start and ntok must be >= 0");
   if ((int64_t)start + ntok > (int64_t)shape->L + shape->T_max)
     return fail(STAR_ERR_CAPACITY, "slots [%d, %d) exceed L + T_max = %d", start, start + ntok, shape->L + shape->T_max);
@@ -234,7 +242,7 @@ int star_phase1_encode(const star_shape* shape, const star_cache* cache, const v
   STAR_REQUIRE_PTR(q, "q");
   STAR_REQUIRE_PTR(k, "k");
   STAR_REQUIRE_PTR(v, "v");
-  STAR_REQUIRE_PTR(pos_ctx, "pos_ctx");
+  STAR_REQUIRE_PTR4(pos_ctx, "pos_ctx");
   STAR_REQUIRE_PTR(out, "out");
   cudaStream_t st = (cudaStream_t)stream;
   const star::CacheView cv = view(shape, cache);
@@ -277,9 +285,9 @@ int star_phase2_partial(const star_shape* shape, const star_cache* cache, const 
   if (!rc) rc = check_cache(shape, cache);
   if (rc) return rc;
   STAR_REQUIRE_PTR(q, "q");
-  STAR_REQUIRE_PTR(q_pos, "q_pos");
+  STAR_REQUIRE_PTR4(q_pos, "q_pos");
   STAR_REQUIRE_PTR(o_part, "o_part");
-  STAR_REQUIRE_PTR(lse_part, "lse_part");
+  STAR_REQUIRE_PTR4(lse_part, "lse_part");
   if ((k == nullptr) != (v == nullptr)) return fail(STAR_ERR_INVALID_ARG, "k and v must both be given or both be NULL");
   if (T <= 0 || T > shape->T_max) return fail(STAR_ERR_INVALID_ARG, "T (%d) must be in [1, T_max=%d]", T, shape->T_max);
   const size_t need = phase2_ws_bytes(shape, T);
@@ -341,9 +349,9 @@ int star_lse_merge(int32_t n_parts, int64_t rows, int32_t d, const float* o_part
   if (n_parts <= 0 || rows < 0) return fail(STAR_ERR_INVALID_ARG, "n_parts must be > 0 and rows >= 0");
   if (d != 64 && d != 128) return fail(STAR_ERR_UNSUPPORTED_SHAPE, "head dim %d is not supported (64 or 128)", d);
   STAR_REQUIRE_PTR(o_part, "o_part");
-  STAR_REQUIRE_PTR(lse_part, "lse_part");
+  STAR_REQUIRE_PTR4(lse_part, "lse_part");
   STAR_REQUIRE_PTR(out, "out");
-  if (lse_out && !aligned16(lse_out)) return fail(STAR_ERR_ALIGNMENT, "lse_out is not 16-byte aligned");
+  if (lse_out && (reinterpret_cast<uintptr_t>(lse_out) & 3u)) return fail(STAR_ERR_ALIGNMENT, "lse_out is not 4-byte aligned");
   cudaError_t e = star::launch_lse_merge(1, n_parts, rows, d, o_part, lse_part, out, true, lse_out, (cudaStream_t)stream);
   return e == cudaSuccess ? STAR_OK : cuda_fail(e, "lse_merge launch");
 }
@@ -357,10 +365,10 @@ int star_decode_step(const star_shape* shape, const star_cache* cache, const voi
   STAR_REQUIRE_PTR(q, "q");
   STAR_REQUIRE_PTR(k, "k");
   STAR_REQUIRE_PTR(v, "v");
-  STAR_REQUIRE_PTR(pos, "pos");
+  STAR_REQUIRE_PTR4(pos, "pos");
   STAR_REQUIRE_PTR(out, "out");
   STAR_REQUIRE_PTR(ws, "ws");
-  if (lse_out && !aligned16(lse_out)) return fail(STAR_ERR_ALIGNMENT, "lse_out is not 16-byte aligned");
+  if (lse_out && (reinterpret_cast<uintptr_t>(lse_out) & 3u)) return fail(STAR_ERR_ALIGNMENT, "lse_out is not 4-byte aligned");
   if (cur_len < 0 || cur_len >= shape->L + shape->T_max)
     return fail(STAR_ERR_CAPACITY, "cur_len %d outside [0, L + T_max = %d)", cur_len, shape->L + shape->T_max);
   const size_t need = decode_ws_bytes(shape);

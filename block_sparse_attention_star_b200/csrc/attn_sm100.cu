@@ -185,13 +185,10 @@ __device__ __forceinline__ void load_q_row(const Params& p, const Item& it, cons
     uint32_t lo[4], hi[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const float2 x1 = unpack_bf16x2(aw[e]);
-      const float2 x2 = unpack_bf16x2(bw[e]);
-      float c0, s0, c1, s1;
-      rope_sincos(r.pos, p.inv_freq[8 * c + 2 * e], c0, s0);
-      rope_sincos(r.pos, p.inv_freq[8 * c + 2 * e + 1], c1, s1);
-      lo[e] = pack_bf16x2(x1.x * c0 - x2.x * s0, x1.y * c1 - x2.y * s1);
-      hi[e] = pack_bf16x2(x2.x * c0 + x1.x * s0, x2.y * c1 + x1.y * s1);
+      double cs[2], sn[2];
+      rope_sincos(r.pos, p.inv_freq[8 * c + 2 * e], cs[0], sn[0]);
+      rope_sincos(r.pos, p.inv_freq[8 * c + 2 * e + 1], cs[1], sn[1]);
+      rope_rotate2(aw[e], bw[e], cs, sn, lo[e], hi[e]);
     }
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
@@ -434,9 +431,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&q_full[wg]);
 
-      float m = -INFINITY, l = 0.f;
+      float m = -INFINITY, l = 0.f, lr = 0.f;
       for (int j = 0; j < nt; ++j) {
-        ok = mbar_wait(&s_full[wg], sph, kDevTimeoutSoftmax);
+        ok = __all_sync(0xffffffffu, mbar_wait(&s_full[wg], sph, kDevTimeoutSoftmax));
         if (!ok) break;
         sph ^= 1;
         tc_fence_after();
@@ -463,21 +460,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           m = m_new;
         }
         const float mu = (m == -INFINITY) ? 0.f : m;
-        // P = 2^(s*scale - m), rounded to bf16; l sums the rounded values.
+        // P = 2^(s*scale - m), rounded to bf16 for the P V product.  Two row sums:
+        // lr of the rounded values normalises O (O = sum P^ V / sum P^ stays a convex
+        // combination of V rows even when one key dominates), lu of the f32 values
+        // gives the log-sum-exp without bf16 rounding.
         uint32_t pk[kKeys / 2];
-        float rs = 0.f;
+        float rs_u = 0.f, rs_r = 0.f;
 #pragma unroll
         for (int c = 0; c < kKeys / 2; ++c) {
           const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * c]), p.scale_log2, -mu));
           const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * c + 1]), p.scale_log2, -mu));
           pk[c] = pack_bf16x2(p0, p1);
-          const float2 r2 = unpack_bf16x2(pk[c]);
-          rs += r2.x + r2.y;
+          rs_u += p0 + p1;
+          rs_r += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xFFFF0000u);
         }
         tmem_st32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
         tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
-        l = l * f + rs;
-        if (rescale && f != 1.f) {
+        l = l * f + rs_u;
+        lr = lr * f + rs_r;
+        // tcgen05.ld/st are warp-collective (.sync.aligned): the whole warp takes
+        // this branch when any of its rows must rescale; the others scale by 1.
+        if (__any_sync(0xffffffffu, f != 1.f)) {
           // O_w holds the products of tiles < j only (its P V for tile j is not
           // issued before p_full), so it can be scaled in place.
 #pragma unroll
@@ -495,11 +498,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&p_full[wg]);
       }
       if (!ok) break;
-      ok = mbar_wait(&o_full[wg], oph, kDevTimeoutSoftmax);
+      ok = __all_sync(0xffffffffu, mbar_wait(&o_full[wg], oph, kDevTimeoutSoftmax));
       if (!ok) break;
       oph ^= 1;
       tc_fence_after();
-      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+      const float inv_l = (lr > 0.f) ? 1.f / lr : 0.f;
       if (MODE == 0) {
         bf16* dst = p.out_bf16 + (((size_t)it.bi * p.L + ri.tok) * p.Hq + ri.head) * D;
 #pragma unroll

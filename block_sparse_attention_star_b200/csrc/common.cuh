@@ -1,10 +1,11 @@
 // Device helpers shared by the Star Attention kernels (sm_100a only).
 //
-// * RoPE angle: the rotation angle pos * inv_freq_j is formed and reduced
-//   modulo 2*pi in float64 (Cody-Waite reduction with 2*pi split into a
-//   float64 head and tail), then sin/cos are taken in float32 on the reduced
-//   angle.  A float32 product pos * inv_freq is off by up to ~0.06 rad at a
-//   million positions, which the float64 angle avoids.
+// * RoPE: the rotation angle pos * inv_freq_j is formed and reduced modulo
+//   2*pi in float64 (Cody-Waite reduction with 2*pi split into a float64 head
+//   and tail), sin/cos and the rotation itself are float64, and each rotated
+//   value is rounded once to bf16.  A float32 angle is off by up to ~0.06 rad
+//   at a million positions; a float32 rotation lands one bf16 step away from
+//   the correctly rounded value often enough to move peaky scores visibly.
 // * mbarrier waits are bounded by the global nanosecond timer: a wait that
 //   runs out records an error code in a device word and returns false, so a
 //   kernel never spins forever.
@@ -39,12 +40,13 @@ extern __device__ int g_device_error;
 
 __device__ __forceinline__ void record_error(int code) { atomicCAS(&g_device_error, 0, code); }
 
-__device__ __forceinline__ void rope_sincos(int pos, double inv_freq, float& c, float& s) {
+// cos and sin of pos * inv_freq in float64 (argument reduced modulo 2*pi first).
+__device__ __forceinline__ void rope_sincos(int pos, double inv_freq, double& c, double& s) {
   const double a = (double)pos * inv_freq;
   const double k = rint(a * kInvTwoPi);
   double r = fma(-k, kTwoPiHi, a);
   r = fma(-k, kTwoPiLo, r);
-  sincosf((float)r, &s, &c);
+  sincos(r, &s, &c);
 }
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
@@ -226,6 +228,25 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t smem_addr, uint32_t
 __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, int a_mn_major, int b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn_major << 15) | ((uint32_t)b_mn_major << 16) |
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2_f64(double lo, double hi) {
+  const __nv_bfloat16 l = __double2bfloat16(lo), h = __double2bfloat16(hi);
+  return (uint32_t)__bfloat16_as_ushort(l) | ((uint32_t)__bfloat16_as_ushort(h) << 16);
+}
+
+// RoPE of two adjacent rotation pairs held as packed bf16x2 words: a holds
+// (x_j, x_{j+1}) of the first half of the head, b holds (x_{j+d/2}, x_{j+1+d/2}).
+// The rotation is done in float64 and each result is rounded once to bf16, so the
+// stored values are the correctly rounded exact rotations.
+__device__ __forceinline__ void rope_rotate2(uint32_t a, uint32_t b, const double (&c)[2], const double (&s)[2],
+                                             uint32_t& lo, uint32_t& hi) {
+  const __nv_bfloat162 av = *reinterpret_cast<const __nv_bfloat162*>(&a);
+  const __nv_bfloat162 bv = *reinterpret_cast<const __nv_bfloat162*>(&b);
+  const double a0 = (double)__bfloat162float(av.x), a1 = (double)__bfloat162float(av.y);
+  const double b0 = (double)__bfloat162float(bv.x), b1 = (double)__bfloat162float(bv.y);
+  lo = pack_bf16x2_f64(a0 * c[0] - b0 * s[0], a1 * c[1] - b1 * s[1]);
+  hi = pack_bf16x2_f64(b0 * c[0] + a0 * s[0], b1 * c[1] + a1 * s[1]);
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {

@@ -71,11 +71,11 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
   for (int e = threadIdx.x; e < G * (D / 2); e += kThreads) {
     const int h = e / (D / 2), j = e % (D / 2);
     const bf16* qr = p.q + ((size_t)bi * p.Hq + g * G + h) * D;
-    const float x1 = __bfloat162float(qr[j]), x2 = __bfloat162float(qr[j + D / 2]);
-    float cs, sn;
+    const double x1 = __bfloat162float(qr[j]), x2 = __bfloat162float(qr[j + D / 2]);
+    double cs, sn;
     rope_sincos(tpos, p.inv_freq[j], cs, sn);
-    qs[h * D + j] = __bfloat162float(__float2bfloat16_rn(x1 * cs - x2 * sn)) * p.scale_log2;
-    qs[h * D + j + D / 2] = __bfloat162float(__float2bfloat16_rn(x2 * cs + x1 * sn)) * p.scale_log2;
+    qs[h * D + j] = __bfloat162float(__double2bfloat16(x1 * cs - x2 * sn)) * p.scale_log2;
+    qs[h * D + j + D / 2] = __bfloat162float(__double2bfloat16(x2 * cs + x1 * sn)) * p.scale_log2;
   }
   __syncthreads();
 

@@ -26,53 +26,52 @@ struct RopeParams {
   double inv_freq[kMaxHalfDim];
 };
 
+// One thread per (sequence, token, 8-pair chunk): the 8 angles are computed once
+// and applied to that chunk of every KV head of the token.
 template <int D>
 __global__ void __launch_bounds__(256) rope_append_kernel(const bf16* __restrict__ k, const bf16* __restrict__ v,
                                                           const int32_t* __restrict__ pos, int B, int ntok, int start,
                                                           int Hkv, bf16* __restrict__ kpool, bf16* __restrict__ vpool,
                                                           const int32_t* __restrict__ page_table, int max_pages,
                                                           int num_pages, int P, const __grid_constant__ RopeParams rp) {
-  constexpr int CH = D / 16;  // threads per (token, head) row: 8 pairs each
-  const long long total = (long long)B * ntok * Hkv * CH;
+  constexpr int CH = D / 16;
+  const long long total = (long long)B * ntok * CH;
   for (long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x; gid < total;
        gid += (long long)gridDim.x * blockDim.x) {
     const int c = (int)(gid % CH);
-    long long r = gid / CH;
-    const int h = (int)(r % Hkv);
-    r /= Hkv;
+    const long long r = gid / CH;
     const int t = (int)(r % ntok);
     const int bi = (int)(r / ntok);
-    const size_t src = (((size_t)bi * ntok + t) * Hkv + h) * D;
     const int slot_abs = start + t;
     const int page = page_table[(size_t)bi * max_pages + slot_abs / P];
     if (page < 0 || page >= num_pages) {
       record_error(kDevBadPage);
       continue;
     }
-    const size_t dst = (((size_t)page * Hkv + h) * P + (slot_abs % P)) * D;
     const int p_t = pos[(size_t)bi * ntok + t];
-
-    const uint4 a = __ldg(reinterpret_cast<const uint4*>(k + src + 8 * c));
-    const uint4 bq = __ldg(reinterpret_cast<const uint4*>(k + src + D / 2 + 8 * c));
-    const uint32_t* aw = reinterpret_cast<const uint32_t*>(&a);
-    const uint32_t* bw = reinterpret_cast<const uint32_t*>(&bq);
-    uint32_t lo[4], hi[4];
+    double cs[4][2], sn[4][2];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const float2 x1 = unpack_bf16x2(aw[e]);
-      const float2 x2 = unpack_bf16x2(bw[e]);
-      float c0, s0, c1, s1;
-      rope_sincos(p_t, rp.inv_freq[8 * c + 2 * e], c0, s0);
-      rope_sincos(p_t, rp.inv_freq[8 * c + 2 * e + 1], c1, s1);
-      lo[e] = pack_bf16x2(x1.x * c0 - x2.x * s0, x1.y * c1 - x2.y * s1);
-      hi[e] = pack_bf16x2(x2.x * c0 + x1.x * s0, x2.y * c1 + x1.y * s1);
+      rope_sincos(p_t, rp.inv_freq[8 * c + 2 * e], cs[e][0], sn[e][0]);
+      rope_sincos(p_t, rp.inv_freq[8 * c + 2 * e + 1], cs[e][1], sn[e][1]);
     }
-    *reinterpret_cast<uint4*>(kpool + dst + 8 * c) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-    *reinterpret_cast<uint4*>(kpool + dst + D / 2 + 8 * c) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-    // V: the same thread copies the two 16-byte chunks at the same offsets.
-    *reinterpret_cast<uint4*>(vpool + dst + 8 * c) = __ldg(reinterpret_cast<const uint4*>(v + src + 8 * c));
-    *reinterpret_cast<uint4*>(vpool + dst + D / 2 + 8 * c) =
-        __ldg(reinterpret_cast<const uint4*>(v + src + D / 2 + 8 * c));
+    for (int h = 0; h < Hkv; ++h) {
+      const size_t src = (((size_t)bi * ntok + t) * Hkv + h) * D;
+      const size_t dst = (((size_t)page * Hkv + h) * P + (slot_abs % P)) * D;
+      const uint4 a = __ldg(reinterpret_cast<const uint4*>(k + src + 8 * c));
+      const uint4 bq = __ldg(reinterpret_cast<const uint4*>(k + src + D / 2 + 8 * c));
+      const uint32_t* aw = reinterpret_cast<const uint32_t*>(&a);
+      const uint32_t* bw = reinterpret_cast<const uint32_t*>(&bq);
+      uint32_t lo[4], hi[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) rope_rotate2(aw[e], bw[e], cs[e], sn[e], lo[e], hi[e]);
+      *reinterpret_cast<uint4*>(kpool + dst + 8 * c) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      *reinterpret_cast<uint4*>(kpool + dst + D / 2 + 8 * c) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      // V: the same thread copies the two 16-byte chunks at the same offsets.
+      *reinterpret_cast<uint4*>(vpool + dst + 8 * c) = __ldg(reinterpret_cast<const uint4*>(v + src + 8 * c));
+      *reinterpret_cast<uint4*>(vpool + dst + D / 2 + 8 * c) =
+          __ldg(reinterpret_cast<const uint4*>(v + src + D / 2 + 8 * c));
+    }
   }
 }
 
@@ -146,7 +145,7 @@ cudaError_t launch_rope_append(const void* k, const void* v, const int32_t* pos,
   if (ntok <= 0 || B <= 0) return cudaSuccess;
   RopeParams rp;
   for (int j = 0; j < d / 2; ++j) rp.inv_freq[j] = rt.inv_freq[j];
-  const long long work = (long long)B * ntok * Hkv * (d / 16);
+  const long long work = (long long)B * ntok * (d / 16);
   const int grid = grid_for(work, 256);
   if (d == 128) {
     rope_append_kernel<128><<<grid, 256, 0, st>>>(

@@ -16,7 +16,8 @@
  * Conventions for every call below
  *   - One attention layer.  Q, K, V are that layer's projections (pre-RoPE).
  *   - Tensor pointers are DEVICE pointers owned by the caller, contiguous,
- *     16-byte aligned; bf16 means IEEE bfloat16.  Layout is [B, tokens, heads, d]
+ *     16-byte aligned (position-id arrays, LSE arrays and the page table: 4-byte
+ *     aligned); bf16 means IEEE bfloat16.  Layout is [B, tokens, heads, d]
  *     ("bshd") unless stated.  Position ids are int32.
  *   - The library allocates no device memory.  Scratch space is passed in as
  *     `ws` of at least star_workspace_size() bytes.
@@ -47,7 +48,7 @@ enum {
   STAR_OK = 0,
   STAR_ERR_INVALID_ARG = -1,      /* null pointer, negative size, inconsistent shape */
   STAR_ERR_UNSUPPORTED_SHAPE = -2,/* valid but not supported: d not in {64,128}, odd Hq/Hkv, L != n*b, ... */
-  STAR_ERR_ALIGNMENT = -3,        /* a pointer is not 16-byte aligned */
+  STAR_ERR_ALIGNMENT = -3,        /* a pointer is not aligned as stated above */
   STAR_ERR_CAPACITY = -4,         /* page table / pool / workspace too small */
   STAR_ERR_CUDA = -5,             /* a CUDA runtime or driver call failed */
   STAR_ERR_TIMEOUT = -6           /* a kernel gave up a bounded wait (see star_device_status) */

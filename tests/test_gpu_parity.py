@@ -51,11 +51,14 @@ def _full_compare(wl, page_table=None, num_pages=None):
     for bi in range(wl.B):
         k, v = res["cache"].gather(bi, 0, wl.L + wl.T + wl.S)
         ck = np.concatenate([ref["cache_k"][bi], oracle.rope_bf16(h.to64(inp["k_query"][bi]), h.to64(inp["pos_query"][bi]).astype(np.int64), wl.theta)])
-        # roped K: bf16 values of the same fp64 rotation; a value may land one bf16 step away.
+        # Roped K: both sides rotate in float64 and round once to bf16, so the values
+        # agree except where sin/cos differ in the last float64 bit right at a bf16
+        # rounding boundary (expected count ~0); allow a handful of one-step flips.
         kg = h.to64(k[: wl.L + wl.T])
         diff = np.abs(kg - ck)
-        assert np.all(diff <= np.abs(ck) * 2.0 ** -7 + 1e-30), "cache K beyond one bf16 step"
-        assert np.mean(diff > 0) < 1e-3, "cache K differs in too many elements"
+        worst = np.unravel_index(np.argmax(diff), diff.shape)
+        assert np.all(diff <= np.abs(ck) * 2.0 ** -7), f"cache K off at {worst}: gpu {kg[worst]} oracle {ck[worst]}"
+        assert np.count_nonzero(diff) <= 4, f"cache K differs in {np.count_nonzero(diff)} elements"
         assert np.array_equal(h.to64(v[: wl.L]), ref["cache_v"][bi]), "cache V must be a bit-exact copy"
     h.assert_out(res["o_part"], ref["o_part"], "phase2 partial O")
     h.assert_lse(res["lse_part"], ref["lse_part"], "phase2 partial LSE")
