@@ -88,6 +88,7 @@ def lib() -> ctypes.CDLL:
             "star_decode_step": ([P(StarShape), P(StarCache), V, V, V, V, I32, V, V, V, SZ, V], ctypes.c_int),
             "star_device_status": ([V, P(I32)], ctypes.c_int),
             "star_set_trace_events": ([V, V], ctypes.c_int),
+            "star_decode_step_noalloc": ([P(StarShape), P(StarCache), V, V, V, V, I32, V, V, V], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -231,6 +232,14 @@ def star_set_trace_events(start=None, stop=None) -> None:
     def handle(ev):
         return None if ev is None else ctypes.c_void_p(ev.cuda_event)
     _check(lib().star_set_trace_events(handle(start), handle(stop)))
+
+
+def star_decode_step_noalloc(shape, cache: PagedKVCache, q, k, v, pos, cur_len: int, out, lse_out, stream=None):
+    """star_decode_step with the library's built-in scratch instead of a caller workspace."""
+    _check(lib().star_decode_step_noalloc(ctypes.byref(shape), ctypes.byref(cache.c), _ptr(q, "q", torch.bfloat16),
+                                          _ptr(k, "k", torch.bfloat16), _ptr(v, "v", torch.bfloat16),
+                                          _ptr(pos, "pos", torch.int32), cur_len, _ptr(out, "out", torch.bfloat16),
+                                          _ptr(lse_out, "lse_out", torch.float32), _stream(stream)))
 
 
 def star_device_status(stream=None) -> int:

@@ -162,6 +162,10 @@ size_t decode_ws_bytes(const star_shape* s) {
 
 }  // namespace
 
+namespace star {
+int set_last_error(int code, const char* msg) { return fail(code, "%s", msg); }
+}  // namespace star
+
 extern "C" {
 
 const char* star_version(void) { return "star-b200 0.1 (sm_100a)"; }

@@ -76,6 +76,9 @@ int decode_pick_chunk(int B, int Hkv, int G, int n_keys, int num_sms);
 size_t decode_smem_bytes(int d, int G, int chunk);
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t st);
 
+// --- api.cu: the thread-local message read by star_last_error(); returns code ----
+int set_last_error(int code, const char* msg);
+
 // --- device error word ---------------------------------------------------------
 cudaError_t read_and_clear_device_error(int* code, cudaStream_t st);
 

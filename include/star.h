@@ -170,6 +170,25 @@ int star_decode_step(const star_shape* shape, const star_cache* cache, const voi
                      const int32_t* pos, int32_t cur_len, void* out, float* lse_out, void* ws, size_t ws_bytes,
                      star_stream_t stream);
 
+/* star_decode_step without a caller workspace.  The Star Attention pages have no
+ * counterpart to this call: it exists for callers that cannot call cudaMalloc, such
+ * as a serving runtime that reserves all device memory for its own pool at start-up
+ * and forbids allocation afterwards, or a plugin that only receives input and
+ * output buffers from the application hosting it.  Arguments, layouts and results
+ * are those of star_decode_step minus (ws, ws_bytes).
+ * Scratch: a 16 MiB device array built into the library (every GPU that loads the
+ * library holds it until the process exits).  The first call made on a device
+ * looks up that array's device address with cudaGetSymbolAddress, so make that
+ * first call before any stream capture.  All calls share the one array and a call
+ * writes every value it later reads, so nothing has to be cleared between calls,
+ * but calls whose kernels overlap on the GPU (other streams, other threads) race
+ * on it: serialise them.  No device memory is allocated or freed.
+ * Errors: those of star_decode_step, plus CAPACITY when the shape's decode partials
+ * (star_workspace_size(shape, STAR_OP_DECODE, ...)) exceed 16 MiB. */
+int star_decode_step_noalloc(const star_shape* shape, const star_cache* cache, const void* q, const void* k,
+                             const void* v, const int32_t* pos, int32_t cur_len, void* out, float* lse_out,
+                             star_stream_t stream);
+
 /* Tracing: when both are non-NULL (cudaEvent_t handles created by the caller),
  * every later call on this thread records `start_event` on its stream right
  * before launching its main kernel and `stop_event` right after it (Phase 1 and

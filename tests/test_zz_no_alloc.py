@@ -1,0 +1,72 @@
+"""The allocation-free decode entry point agrees with the workspace one.
+
+star_decode_step_noalloc is for callers that cannot call cudaMalloc (a runtime
+whose device memory is all reserved up front, a plugin handed only its input and
+output buffers).  This file is collected last so that, if it fails, every other
+test has already run.  It builds two identical caches, then decodes the same two
+tokens in a row on each: through star_decode_step (caller workspace) and through
+star_decode_step_noalloc (built-in scratch), called through the C ABI.
+"""
+
+import pytest
+import torch
+
+from synth import Workload, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def _prefill(wl, inp, star, harness):
+    shape = harness.shape_of(wl)
+    cache = star.PagedKVCache(shape)
+    out = torch.empty_like(inp["q_ctx"])
+    star.star_phase1_encode(shape, cache, inp["q_ctx"], inp["k_ctx"], inp["v_ctx"], inp["pos_ctx"], out)
+    star.star_kv_append(shape, cache, inp["k_query"], inp["v_query"], inp["pos_query"], wl.L, wl.T)
+    return shape, cache
+
+
+@pytest.mark.parametrize("wl", [
+    Workload("noalloc-d128", B=2, Hq=8, Hkv=2, d=128, L=2048, b=512, T=40, S=2, peaky=True),
+    Workload("noalloc-d64", B=1, Hq=4, Hkv=1, d=64, L=1024, b=256, T=16, S=2, peaky=False),
+])
+def test_noalloc_decode_matches_workspace_decode(wl):
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import block_sparse_attention_star_b200 as star
+    from tests import harness
+    inp = make_inputs(wl, "cuda")
+    shape_a, cache_a = _prefill(wl, inp, star, harness)
+    shape_b, cache_b = _prefill(wl, inp, star, harness)
+    ws = star.workspace(shape_a, star.STAR_OP_DECODE)
+    for s in range(2):
+        cur = wl.L + wl.T + s
+        ref_o = torch.empty((wl.B, 1, wl.Hq, wl.d), dtype=torch.bfloat16, device="cuda")
+        ref_l = torch.empty((wl.B, wl.Hq), dtype=torch.float32, device="cuda")
+        star.star_decode_step(shape_a, cache_a, inp["q_dec"][s], inp["k_dec"][s], inp["v_dec"][s], inp["pos_dec"][s],
+                              cur, ref_o, ref_l, ws)
+        got_o = torch.full_like(ref_o, float("nan"))
+        got_l = torch.full_like(ref_l, float("nan"))
+        star.star_decode_step_noalloc(shape_b, cache_b, inp["q_dec"][s], inp["k_dec"][s], inp["v_dec"][s],
+                                      inp["pos_dec"][s], cur, got_o, got_l)
+        torch.cuda.synchronize()
+        harness.assert_out(got_o, harness.to64(ref_o), f"noalloc decode step {s} O")
+        harness.assert_lse(got_l, harness.to64(ref_l), f"noalloc decode step {s} LSE")
+    assert star.star_device_status() == 0
+
+
+def test_noalloc_rejects_shapes_beyond_its_scratch():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import block_sparse_attention_star_b200 as star
+    from tests import harness
+    big = Workload("noalloc-big", B=8, Hq=64, Hkv=8, d=128, L=1 << 20, b=1 << 17, T=32, S=16, peaky=False)
+    shape = harness.shape_of(big)
+    assert star.star_workspace_size(shape, star.STAR_OP_DECODE) > 16 << 20
+    small = Workload("noalloc-small", B=1, Hq=4, Hkv=1, d=64, L=1024, b=256, T=16, S=2, peaky=False)
+    cache = star.PagedKVCache(harness.shape_of(small))
+    q = torch.zeros((big.B, 1, big.Hq, big.d), dtype=torch.bfloat16, device="cuda")
+    kv = torch.zeros((big.B, 1, big.Hkv, big.d), dtype=torch.bfloat16, device="cuda")
+    pos = torch.zeros(big.B, dtype=torch.int32, device="cuda")
+    with pytest.raises(star.StarError) as e:
+        star.star_decode_step_noalloc(shape, cache, q, kv, kv, pos, 0, q, None)
+    assert e.value.code == star.STAR_ERR_CAPACITY and "16777216" in str(e.value)
