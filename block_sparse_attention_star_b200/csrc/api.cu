@@ -123,8 +123,9 @@ float scale_log2(const star_shape* s) { return (float)(1.4426950408889634 / std:
     if (!aligned16(p)) return fail(STAR_ERR_ALIGNMENT, "%s is not 16-byte aligned", name); \
   } while (0)
 
-// Phase 2 splits each block into chunks_per_block parts so the grid fills the
-// GPU; the smallest divisor of b/128 that gives >= 2 items per SM.
+// Phase 2 splits each block into chunks_per_block parts so the persistent grid
+// fills the GPU with long items: the largest divisor of b/128 that keeps the item
+// count within one wave (one item per SM); 1 if even that exceeds a wave.
 int phase2_chunks_per_block(const star_shape* s, int T) {
   const int G = s->Hq / s->Hkv;
   int TQ = 1;
@@ -134,11 +135,11 @@ int phase2_chunks_per_block(const star_shape* s, int T) {
   const int NHT = (G + HT - 1) / HT;
   const int npairs = (NTT * NHT + 1) / 2;
   const int64_t base = (int64_t)s->n * s->B * s->Hkv * npairs;
-  const int64_t need = (2LL * num_sms() + base - 1) / base;
   const int nb = s->b / 128;
+  int best = 1;
   for (int c = 1; c <= nb; ++c)
-    if (nb % c == 0 && c >= need) return c;
-  return nb;
+    if (nb % c == 0 && base * c <= num_sms()) best = c;
+  return best;
 }
 
 size_t phase2_ws_bytes(const star_shape* s, int T) {

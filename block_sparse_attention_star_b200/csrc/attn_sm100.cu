@@ -53,6 +53,9 @@ constexpr int kRows = 128;        // rows per Q tile (UMMA M)
 constexpr int kKeys = 128;        // keys per K/V tile (UMMA N of QK^T, K of PV)
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
+constexpr uint32_t kRegsCtl = 56;
+constexpr uint32_t kRegsSoftmax = 224;
+static_assert(128 * kRegsCtl + 256 * kRegsSoftmax <= kThreads * 168, "register split exceeds the launch budget");
 
 struct Params {
   const bf16* q;
@@ -262,6 +265,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
+  // Registers: the producer/MMA warpgroup (warps 0-3) needs few, the softmax
+  // warpgroups hold a 128-score row each.  128 x kRegsCtl + 256 x kRegsSoftmax
+  // stays within the 384 x 168 registers the CTA is launched with.
+  if (warp < 4) {
+  setmaxnreg_dec<kRegsCtl>();
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
@@ -410,7 +418,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(drain, 0, kDevTimeoutMma);
       }
     }
-  } else if (warp >= 4) {
+  }
+  } else {
+    setmaxnreg_inc<kRegsSoftmax>();
     // ------------------------------------------------------------------ softmax warpgroups
     const int wg = (warp - 4) / 4;
     const int wq = warp % 4;
@@ -423,10 +433,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
 
     for (int idx = blockIdx.x; idx < p.num_items && ok; idx += gridDim.x) {
-      const Item it = decode_item<MODE>(p, idx);
-      const int nt = it.a_tiles + it.b_tiles;
-      const RowInfo ri = row_info<MODE>(p, it, wg, row);
-      load_q_row<D>(p, it, ri, sQ, row);
+      int nt, a_tiles, a_start, b_start, cache_idx;
+      {
+        const Item it = decode_item<MODE>(p, idx);
+        const RowInfo ri = row_info<MODE>(p, it, wg, row);
+        load_q_row<D>(p, it, ri, sQ, row);
+        nt = it.a_tiles + it.b_tiles;
+        a_tiles = it.a_tiles;
+        a_start = it.a_start;
+        b_start = it.b_start;
+        cache_idx = ri.cache_idx;
+      }
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&q_full[wg]);
@@ -441,17 +458,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
         tmem_ld_wait();
-        const int k0 = tile_key0(it, j);
-        if (k0 + kKeys - 1 > ri.cache_idx) {
-          const int lim = ri.cache_idx - k0;  // keys k0 + c with c > lim are not visible
+        const int k0 = j < a_tiles ? a_start + j * kKeys : b_start + (j - a_tiles) * kKeys;
+        if (k0 + kKeys - 1 > cache_idx) {
+          const int lim = cache_idx - k0;  // keys k0 + c with c > lim are not visible
 #pragma unroll
           for (int c = 0; c < kKeys; ++c)
             if (c > lim) sr[c] = __float_as_uint(-INFINITY);
         }
-        // Row max of the raw scores (scale > 0 commutes with max).
-        float mt = __uint_as_float(sr[0]);
+        // Row max of the raw scores (scale > 0 commutes with max); 4 independent chains.
+        float mx[4];
 #pragma unroll
-        for (int c = 1; c < kKeys; ++c) mt = fmaxf(mt, __uint_as_float(sr[c]));
+        for (int e = 0; e < 4; ++e) mx[e] = __uint_as_float(sr[e]);
+#pragma unroll
+        for (int c = 4; c < kKeys; ++c) mx[c % 4] = fmaxf(mx[c % 4], __uint_as_float(sr[c]));
+        const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
         const float m_new = fmaxf(m, mt * p.scale_log2);
         float f = 1.f;
         const bool rescale = m_new > m + kRescaleThreshold;
@@ -464,18 +484,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         // lr of the rounded values normalises O (O = sum P^ V / sum P^ stays a convex
         // combination of V rows even when one key dominates), lu of the f32 values
         // gives the log-sum-exp without bf16 rounding.
-        uint32_t pk[kKeys / 2];
-        float rs_u = 0.f, rs_r = 0.f;
+        // One pair in four takes 2^x on the FMA pipe, the rest on the MUFU unit, so
+        // the exponentials of both warpgroups fit under the tensor time.  P is
+        // written to TMEM in two 32-column halves so the score registers free early.
+        float su[2] = {0.f, 0.f}, sq[2] = {0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < kKeys / 2; ++c) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * c]), p.scale_log2, -mu));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * c + 1]), p.scale_log2, -mu));
-          pk[c] = pack_bf16x2(p0, p1);
-          rs_u += p0 + p1;
-          rs_r += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xFFFF0000u);
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const int cc = half * 32 + c;
+            const float x0 = fmaf(__uint_as_float(sr[2 * cc]), p.scale_log2, -mu);
+            const float x1 = fmaf(__uint_as_float(sr[2 * cc + 1]), p.scale_log2, -mu);
+            float p0, p1;
+            if ((c & 3) == 3) {
+              p0 = exp2_poly3(x0);
+              p1 = exp2_poly3(x1);
+            } else {
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
+            pk[c] = pack_bf16x2(p0, p1);
+            su[c & 1] += p0 + p1;
+            sq[c & 1] += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xFFFF0000u);
+          }
+          tmem_st32(tS + half * 32, pk);
         }
-        tmem_st32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-        tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+        const float rs_u = su[0] + su[1];
+        const float rs_r = sq[0] + sq[1];
         l = l * f + rs_u;
         lr = lr * f + rs_r;
         // tcgen05.ld/st are warp-collective (.sync.aligned): the whole warp takes
@@ -502,6 +538,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       oph ^= 1;
       tc_fence_after();
+      const Item it = decode_item<MODE>(p, idx);
+      const RowInfo ri = row_info<MODE>(p, it, wg, row);
       const float inv_l = (lr > 0.f) ? 1.f / lr : 0.f;
       if (MODE == 0) {
         bf16* dst = p.out_bf16 + (((size_t)it.bi * p.L + ri.tok) * p.Hq + ri.head) * D;
