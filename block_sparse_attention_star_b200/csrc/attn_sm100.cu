@@ -480,38 +480,32 @@ __global__ void __launch_bounds__(kThreads, 1)
           m = m_new;
         }
         const float mu = (m == -INFINITY) ? 0.f : m;
-        // P = 2^(s*scale - m), rounded to bf16 for the P V product.  Two row sums:
-        // lr of the rounded values normalises O (O = sum P^ V / sum P^ stays a convex
-        // combination of V rows even when one key dominates), lu of the f32 values
-        // gives the log-sum-exp without bf16 rounding.
-        // One pair in four takes 2^x on the FMA pipe, the rest on the MUFU unit, so
-        // the exponentials of both warpgroups fit under the tensor time.  P is
-        // written to TMEM in two 32-column halves so the score registers free early.
-        float su[2] = {0.f, 0.f}, sq[2] = {0.f, 0.f};
+        // P = 2^(s*scale - m) (exponent arguments two at a time), rounded to bf16 for
+        // the P V product; l sums the f32 values (the log-sum-exp needs no bf16
+        // rounding in it).  P is written to TMEM in two 32-column halves.
+        const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
+        const uint64_t nm2 = f2_pack(-mu, -mu);
+        float su[2] = {0.f, 0.f};
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t pk[32];
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
             const int cc = half * 32 + c;
-            const float x0 = fmaf(__uint_as_float(sr[2 * cc]), p.scale_log2, -mu);
-            const float x1 = fmaf(__uint_as_float(sr[2 * cc + 1]), p.scale_log2, -mu);
-            float p0, p1;
-            if ((c & 3) == 3) {
-              p0 = exp2_poly3(x0);
-              p1 = exp2_poly3(x1);
-            } else {
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
-            }
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * cc]), __uint_as_float(sr[2 * cc + 1])), sc2, nm2), x0, x1);
+            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
             pk[c] = pack_bf16x2(p0, p1);
             su[c & 1] += p0 + p1;
-            sq[c & 1] += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xFFFF0000u);
           }
           tmem_st32(tS + half * 32, pk);
         }
         const float rs_u = su[0] + su[1];
-        const float rs_r = sq[0] + sq[1];
+        // O is normalised by the sum of the bf16-rounded P so that it stays a convex
+        // combination of V rows when one key dominates; the rounding that matters
+        // there is the largest P's, so its error is added to the f32 sum.
+        const float pmax = ex2_approx(fmaf(mt, p.scale_log2, -mu));
+        const float rs_r = rs_u + (__bfloat162float(__float2bfloat16_rn(pmax)) - pmax);
         l = l * f + rs_u;
         lr = lr * f + rs_r;
         // tcgen05.ld/st are warp-collective (.sync.aligned): the whole warp takes

@@ -249,23 +249,20 @@ __device__ __forceinline__ void rope_rotate2(uint32_t a, uint32_t b, const doubl
   hi = pack_bf16x2_f64(b0 * c[0] + a0 * s[0], b1 * c[1] + a1 * s[1]);
 }
 
-// 2^x on the FMA pipe, for x <= 8 (the softmax's lazily rescaled exponents).
-// x = j + f with j = round(x), f in [-1/2, 1/2]; 2^f by a cubic fitted to minimise
-// the relative error on [-1/2, 1/2] (Lawson-reweighted least squares on Chebyshev
-// nodes, coefficients computed for this kernel; max relative error 7.5e-5 in
-// float32 Horner form, below the bf16 rounding of P and far below the LSE
-// tolerance); 2^j is added to the exponent field.  Inputs below -126 return 2^-126.
-__device__ __forceinline__ float exp2_poly3(float x) {
-  x = fmaxf(x, -126.0f);
-  const float t = x + 12582912.0f;   // 1.5 * 2^23: rounds x to an integer in t's low bits
-  const float r = t - 12582912.0f;
-  const float f = x - r;
-  const float p = fmaf(fmaf(fmaf(0.055171653628349304f, f, 0.2426111251115799f), f, 0.6932609677314758f), f,
-                       0.9999280571937561f);
-  const int j = __float_as_int(t) - 0x4B400000;
-  return __int_as_float(__float_as_int(p) + (j << 23));
+// Packed float pairs (sm_100 f32x2 arithmetic): two lanes of work per instruction.
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
 }
-
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
 // Register reallocation for a whole warpgroup (all 128 threads must execute it).
 template <uint32_t N>
 __device__ __forceinline__ void setmaxnreg_inc() {
