@@ -37,7 +37,7 @@ def build(force: bool = False, ptxas_verbose: bool = False) -> str:
     cmd = [
         nvcc_path(),
         "-gencode", "arch=compute_100a,code=sm_100a",
-        "-O3", "-lineinfo", "-std=c++17", "-rdc=true",
+        "-O3", "-lineinfo", "-std=c++17",
         "-Xcompiler", "-fPIC,-O2", "-shared",
         "-I", os.path.join(ROOT, "include"),
         "-o", LIB + ".tmp",

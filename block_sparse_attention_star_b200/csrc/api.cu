@@ -420,7 +420,15 @@ int star_set_trace_events(void* start_event, void* stop_event) {
 
 int star_device_status(star_stream_t stream, int32_t* status_out) {
   int code = 0;
-  cudaError_t e = star::read_and_clear_device_error(&code, (cudaStream_t)stream);
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  cudaError_t (*readers[])(int*) = {star::read_and_clear_error_attn, star::read_and_clear_error_decode,
+                                   star::read_and_clear_error_rope};
+  for (auto rd : readers) {
+    if (e != cudaSuccess) break;
+    int c = 0;
+    e = rd(&c);
+    if (code == 0) code = c;
+  }
   if (status_out) *status_out = code;
   if (e != cudaSuccess) return cuda_fail(e, "device status");
   if (code == star::kDevBadPage) return fail(STAR_ERR_CAPACITY, "a page-table entry was outside [0, num_pages)");

@@ -44,8 +44,6 @@
 
 namespace star {
 
-__device__ int g_device_error = 0;
-
 namespace {
 
 constexpr int kThreads = 384;
@@ -53,9 +51,14 @@ constexpr int kRows = 128;        // rows per Q tile (UMMA M)
 constexpr int kKeys = 128;        // keys per K/V tile (UMMA N of QK^T, K of PV)
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
-constexpr uint32_t kRegsCtl = 56;
-constexpr uint32_t kRegsSoftmax = 224;
-static_assert(128 * kRegsCtl + 256 * kRegsSoftmax <= kThreads * 168, "register split exceeds the launch budget");
+// Per-warpgroup register budgets (setmaxnreg), chosen so neither role spills;
+// 128 x ctl + 256 x softmax must stay within the 384 x 168 registers of the launch.
+template <int D>
+struct RegSplit {
+  static constexpr uint32_t kCtl = (D == 128) ? 104 : 72;
+  static constexpr uint32_t kSoftmax = (D == 128) ? 200 : 216;
+  static_assert(128 * kCtl + 256 * kSoftmax <= kThreads * 168, "register split exceeds the launch budget");
+};
 
 struct Params {
   const bf16* q;
@@ -265,11 +268,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  // Registers: the producer/MMA warpgroup (warps 0-3) needs few, the softmax
-  // warpgroups hold a 128-score row each.  128 x kRegsCtl + 256 x kRegsSoftmax
-  // stays within the 384 x 168 registers the CTA is launched with.
+  // Registers: the producer/MMA warpgroup (warps 0-3) needs fewer than the softmax
+  // warpgroups, which hold a 128-score row each (RegSplit).
   if (warp < 4) {
-  setmaxnreg_dec<kRegsCtl>();
+  setmaxnreg_dec<RegSplit<D>::kCtl>();
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
@@ -420,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   } else {
-    setmaxnreg_inc<kRegsSoftmax>();
+    setmaxnreg_inc<RegSplit<D>::kSoftmax>();
     // ------------------------------------------------------------------ softmax warpgroups
     const int wg = (warp - 4) / 4;
     const int wq = warp % 4;
@@ -697,13 +699,6 @@ cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t st, const char** 
   }
 }
 
-cudaError_t read_and_clear_device_error(int* code, cudaStream_t st) {
-  cudaError_t e = cudaStreamSynchronize(st);
-  if (e != cudaSuccess) return e;
-  e = cudaMemcpyFromSymbol(code, g_device_error, sizeof(int));
-  if (e != cudaSuccess) return e;
-  const int zero = 0;
-  return cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
-}
+cudaError_t read_and_clear_error_attn(int* code) { return read_and_clear_tu_error(code); }
 
 }  // namespace star

@@ -28,7 +28,10 @@ constexpr double kTwoPiLo = 2.4492935982947064e-16;
 constexpr double kInvTwoPi = 0.15915494309189535;
 constexpr int kMaxHalfDim = 64;   // head_dim <= 128
 
-// Device-side error word (first error wins); read and cleared by the host.
+// Device-side error word (first error wins), one per translation unit: the
+// library is built without relocatable device code so that ptxas can apply the
+// per-warpgroup register budgets of setmaxnreg; each kernel file exposes its
+// word through a host reader (internal.h) and star_device_status combines them.
 enum DeviceError : int {
   kDevOk = 0,
   kDevTimeoutProducer = 1,
@@ -36,9 +39,18 @@ enum DeviceError : int {
   kDevTimeoutSoftmax = 3,
   kDevBadPage = 4,
 };
-extern __device__ int g_device_error;
+static __device__ int g_device_error = 0;
 
 __device__ __forceinline__ void record_error(int code) { atomicCAS(&g_device_error, 0, code); }
+
+// Host: read this translation unit's error word and clear it (the caller has
+// synchronised the stream).
+static inline cudaError_t read_and_clear_tu_error(int* code) {
+  cudaError_t e = cudaMemcpyFromSymbol(code, g_device_error, sizeof(int));
+  if (e != cudaSuccess) return e;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+}
 
 // cos and sin of pos * inv_freq in float64 (argument reduced modulo 2*pi first).
 __device__ __forceinline__ void rope_sincos(int pos, double inv_freq, double& c, double& s) {

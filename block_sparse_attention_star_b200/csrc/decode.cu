@@ -380,6 +380,8 @@ size_t decode_smem_bytes(int d, int G, int chunk) {
   }
 }
 
+cudaError_t read_and_clear_error_decode(int* code) { return read_and_clear_tu_error(code); }
+
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t st) {
   DecParams p;
   p.q = reinterpret_cast<const bf16*>(a.q);

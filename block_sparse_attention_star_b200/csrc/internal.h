@@ -79,7 +79,9 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t st);
 // --- api.cu: the thread-local message read by star_last_error(); returns code ----
 int set_last_error(int code, const char* msg);
 
-// --- device error word ---------------------------------------------------------
-cudaError_t read_and_clear_device_error(int* code, cudaStream_t st);
+// --- device error words (one per kernel file; call after synchronising) ------
+cudaError_t read_and_clear_error_attn(int* code);
+cudaError_t read_and_clear_error_decode(int* code);
+cudaError_t read_and_clear_error_rope(int* code);
 
 }  // namespace star

@@ -140,6 +140,8 @@ int grid_for(long long work, int threads) {
 
 }  // namespace
 
+cudaError_t read_and_clear_error_rope(int* code) { return read_and_clear_tu_error(code); }
+
 cudaError_t launch_rope_append(const void* k, const void* v, const int32_t* pos, int B, int ntok, int start, int Hkv,
                                int d, const CacheView& c, const RopeTable& rt, cudaStream_t st) {
   if (ntok <= 0 || B <= 0) return cudaSuccess;
