@@ -168,6 +168,41 @@ class StarRun:
             s.star_set_trace_events(None, None)
 
 
+def measured_traffic(B: int, L: int):
+    """DRAM bytes of one Phase-1 launch from the committed ncu record, scaled by context tokens;
+    None when the kernel sources changed since the counters were taken."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "attn_phase1_traffic.json")) as f:
+            rec = json.load(f)
+        h = hashlib.sha256(b"".join(open(os.path.join(ROOT, src), "rb").read() for src in rec["sources"])).hexdigest()
+        if h != rec["source_sha256"]:
+            return None
+        return rec["dram_bytes_per_context_token"] * B * L
+    except Exception:
+        return None
+
+
+def rank_workload(name: str, rank: int):
+    """The workload rank `rank` runs: the same shapes, its own seed (independent sequences)."""
+    wl0 = get_config(name)
+    return dataclasses.replace(wl0, seed=wl0.seed + rank)
+
+
+def max_over_ranks(value: float, device) -> float:
+    """The maximum of `value` over all ranks (the job's time is its slowest rank's)."""
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world: int, B: int, L: int, ms_per_step: float) -> float:
+    """Whole-job context tokens per second: every rank encodes B sequences of L tokens per step."""
+    return world * B * L / (ms_per_step * 1e-3)
+
+
 def _ev():
     return torch.cuda.Event(enable_timing=True)
 
@@ -218,8 +253,7 @@ def run_star(args, rank, world, local_rank):
     peaks = load_peaks()
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    wl0 = get_config(args.config)
-    wl = dataclasses.replace(wl0, seed=wl0.seed + rank)
+    wl = rank_workload(args.config, rank)
     run = StarRun(wl, dev)
     star = run.star
 
@@ -245,11 +279,7 @@ def run_star(args, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     status = star.star_device_status()
-    ms_total = t0.elapsed_time(t1)
-    ms_tensor = torch.tensor([ms_total], device=dev)
-    if world > 1:
-        dist.all_reduce(ms_tensor, op=dist.ReduceOp.MAX)
-    ms_step = float(ms_tensor.item()) / K
+    ms_step = max_over_ranks(t0.elapsed_time(t1), dev) / K
 
     p1_ms = statistics.mean(e["p1"][0].elapsed_time(e["p1"][1]) for e in evs)
     p2_ms = statistics.mean(e["p2"][0].elapsed_time(e["p2"][1]) for e in evs)
@@ -264,7 +294,7 @@ def run_star(args, rank, world, local_rank):
     if not args.no_e2e:
         e2e = run_e2e(run, K, max(3, args.warmup), world)
 
-    value = world * wl.B * wl.L / (ms_step * 1e-3)
+    value = job_value(world, wl.B, wl.L, ms_step)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": max(3, args.warmup),
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -279,7 +309,7 @@ def run_star(args, rank, world, local_rank):
         "decode": {"us_per_step": 1e3 * statistics.mean(dec_call_ms), "kernel_us": 1e3 * statistics.mean(dec_kernel_ms),
                    "bytes_per_step": dec_bytes, "kernel_gbs": dec_gbs, "frac_hbm": dec_gbs / peaks["hbm_gbs"]},
         "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
-                     "frac": tflops / peaks["bf16_sustained"], "traffic": None,
+                     "frac": tflops / peaks["bf16_sustained"], "traffic": measured_traffic(wl.B, wl.L),
                      "kernel": f"star_attn_kernel<{wl.d},0> (Phase 1)", "flop_per_launch": flops,
                      "peak_source": peaks["kind"] + " bf16 sustained"},
         "gpu_launches": run.launches_per_step * K,
@@ -324,11 +354,9 @@ def run_e2e(run, K, W, world):
         one()
     t1.record()
     torch.cuda.synchronize()
-    ms = torch.tensor([t0.elapsed_time(t1) / K], device=run.dev)
-    if world > 1:
-        dist.all_reduce(ms, op=dist.ReduceOp.MAX)
-    return {"value": world * wl.B * wl.L / (float(ms.item()) * 1e-3), "unit": UNIT,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": float(ms.item())}
+    ms = max_over_ranks(t0.elapsed_time(t1) / K, run.dev)
+    return {"value": job_value(world, wl.B, wl.L, ms), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms}
 
 
 # ---------------------------------------------------------------------------

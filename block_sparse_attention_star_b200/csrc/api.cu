@@ -381,8 +381,7 @@ int star_decode_step(const star_shape* shape, const star_cache* cache, const voi
   cudaStream_t st = (cudaStream_t)stream;
   const star::CacheView cv = view(shape, cache);
   const star::RopeTable rt = rope_table(shape);
-  cudaError_t e = star::launch_rope_append(k, v, pos, shape->B, 1, cur_len, shape->Hkv, shape->d, cv, rt, st);
-  if (e != cudaSuccess) return cuda_fail(e, "decode kv append");
+  cudaError_t e;
   const int chunk = decode_chunk(shape);
   const int n_keys = cur_len + 1;
   const int nch = star::decode_num_chunks(n_keys, chunk);
@@ -394,6 +393,8 @@ int star_decode_step(const star_shape* shape, const star_cache* cache, const voi
   a.Hkv = shape->Hkv;
   a.d = shape->d;
   a.q = q;
+  a.k_new = k;
+  a.v_new = v;
   a.pos = pos;
   a.n_keys = n_keys;
   a.chunk = chunk;

@@ -8,19 +8,24 @@
 // chunks (a finer partition than blocks; the merge is associative, so chunk
 // partials merge to the same result as per-block partials).  One CTA per
 // (chunk, KV head, sequence) serves all G query heads of the group, so each K/V
-// byte is fetched once for G heads.  The grid is sized to two CTAs per SM, one
-// wave.
+// byte is fetched once for G heads.  The grid is one wave of kCtasPerSm CTAs per SM.
 //
-// CTA: warp 8 is the TMA producer (64-key K and V tiles, 128-byte swizzle, a
-// 3- or 2-stage ring, no multicast); warps 0-7 compute, per tile:
-//   1. QK: thread (key pair kp, dim eighth e) reads 16 dims of keys kp and kp+32
-//      (swizzled, conflict-free) and the G query vectors' same 16 dims (shared-
-//      memory broadcast), and writes G x 2 partial dot products.
-//   2. softmax: warp h owns head h: sums the 8 partials, masks keys past the
-//      cache, and updates its running max / sum (online softmax, base 2).
-//   3. PV: warp w accumulates keys [8w, 8w+8) into its lanes' 4 dims x G heads.
-// At the end the 8 warps' accumulators are reduced and the chunk's normalised
-// O and natural-log LSE are written for the merge kernel.
+// The CTA that owns the last chunk of a (sequence, KV head) first appends the new
+// token: RoPE(k) (float64 rotation, one bf16 rounding, like star_kv_append) and v
+// go to cache slot n_keys - 1, made visible to its own TMA loads by a proxy fence.
+//
+// CTA: warp 8 is the TMA producer (64-key K and V tiles, 128-byte swizzle, an
+// NST-stage ring, no multicast); warps 0-7 compute.  Warp w owns keys
+// [8w, 8w + 8) of every tile and keeps its own online softmax (running max m and
+// sum l per head, base 2), so there is no CTA barrier per tile:
+//   QK: lane = (key kk = lane / 4, quarter = lane % 4); it dots its quarter of
+//       the key with the same quarter of the G query vectors (shared-memory
+//       broadcast from a padded layout); two shuffles finish the dot products.
+//   softmax: max and sum over the warp's 8 keys by shuffles; P goes to a small
+//       per-warp shared buffer.
+//   PV: lane owns d/32 dims of the G outputs and accumulates the 8 keys.
+// At the end the 8 warps' (m, l, O) are combined and the chunk's normalised O and
+// natural-log LSE are written for the merge kernel.
 #include "common.cuh"
 #include "internal.h"
 
@@ -29,20 +34,20 @@
 namespace star {
 namespace {
 
-constexpr int kCompute = 256;          // compute threads (8 warps)
-constexpr int kThreads = kCompute + 32; // + producer warp
+constexpr int kCompute = 256;            // compute threads (8 warps)
+constexpr int kThreads = kCompute + 32;  // + producer warp
 constexpr int kTileKeys = 64;
-constexpr int kCtasPerSm = 2;
 constexpr int kMaxChunk = 1 << 16;
-
-template <int G>
-struct DecCfg {
-  static constexpr int NST = (G <= 4) ? 3 : 2;
-};
+constexpr int kCtasPerSm = 2;
+constexpr int kStages = 3;
 
 struct DecParams {
-  const bf16* q;
-  const int32_t* pos;
+  const bf16* q;       // [B][Hq][D]
+  const bf16* k_new;   // [B][Hkv][D]: the token appended at slot n_keys - 1
+  const bf16* v_new;
+  bf16* kpool;
+  bf16* vpool;
+  const int32_t* pos;  // [B]
   const int32_t* page_table;
   float* o_ws;
   float* lse_ws;
@@ -54,17 +59,16 @@ struct DecParams {
 
 template <int D, int G>
 struct DecSmem {
-  static constexpr int NST = DecCfg<G>::NST;
+  static constexpr int NST = kStages;
+  static constexpr int QPAD = D / 4 + 4;                  // floats per (head, quarter) row
   static constexpr int kTile = kTileKeys * D * 2;         // one K or V tile
-  static constexpr int kStage = 2 * kTile;                 // K then V
-  static constexpr int kQ = NST * kStage;                  // f32 [G][D]
-  static constexpr int kPart = kQ + G * D * 4;             // f32 [8][G][64]
-  static constexpr int kP = kPart + 8 * G * kTileKeys * 4; // f32 [64][G]
-  static constexpr int kStat = kP + kTileKeys * G * 4;     // f32 alpha[G], m[G], l[G]
-  static constexpr int kBar = ((kStat + 3 * G * 4) + 7) / 8 * 8;
+  static constexpr int kStage = 2 * kTile;                // K then V
+  static constexpr int kQ = NST * kStage;                 // f32 [G][4][QPAD]
+  static constexpr int kP = kQ + G * 4 * QPAD * 4;        // f32 [8 warps][8 keys][G]
+  static constexpr int kBar = (kP + 8 * 8 * G * 4 + 7) / 8 * 8;
   static constexpr int kEnd = kBar + 2 * NST * 8;
   static constexpr int kBytes = kEnd + 1024;
-  static_assert(8 * G * D * 4 <= NST * kStage, "final reduction must fit in the stage buffers");
+  static_assert(8 * G * (D + 2) * 4 <= NST * kStage, "final combine must fit in the stage buffers");
 };
 
 // Byte offset of element (key, d) in a swizzled 64-key tile: 64-element d halves
@@ -76,18 +80,7 @@ __device__ __forceinline__ int tile_off(int key, int d) {
 
 __device__ __forceinline__ void bar_compute() { asm volatile("bar.sync 1, %0;" ::"n"(kCompute) : "memory"); }
 
-// Barrier over the compute warps that also returns whether `v` holds in all of them,
-// so every warp takes the same give-up decision.
-__device__ __forceinline__ bool bar_compute_all(bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, 1, %2, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)v), "n"(kCompute)
-      : "memory");
-  return r != 0;
-}
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 
 template <int D, int G>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
@@ -95,12 +88,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                   const __grid_constant__ DecParams p) {
   using S = DecSmem<D, G>;
   constexpr int NST = S::NST;
+  constexpr int QPAD = S::QPAD;
+  constexpr int DQ = D / 4;    // dims per quarter (QK)
+  constexpr int DPL = D / 32;  // dims per lane (PV)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* qs = reinterpret_cast<float*>(smem + S::kQ);
-  float* part = reinterpret_cast<float*>(smem + S::kPart);
-  float* ps = reinterpret_cast<float*>(smem + S::kP);
-  float* stat = reinterpret_cast<float*>(smem + S::kStat);
+  float* ps_all = reinterpret_cast<float*>(smem + S::kP);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBar);
   uint64_t* empty = full + NST;
 
@@ -111,25 +105,54 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   const int k_end = min(k_begin + p.chunk, p.n_keys);
   const int ntiles = (k_end - k_begin + kTileKeys - 1) / kTileKeys;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int tpos = p.pos[bi];
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], 8);
     }
     fence_barrier_init();
   }
+  // The owner of the last chunk appends the new token (head g) before any load.
+  if (c == p.nchunks - 1) {
+    const int slot_abs = p.n_keys - 1;
+    const int page = p.page_table[(size_t)bi * p.max_pages + slot_abs / p.P];
+    if (page < 0 || page >= p.num_pages) {
+      if (threadIdx.x == 0) record_error(kDevBadPage);
+    } else {
+      const size_t dst = (((size_t)page * p.Hkv + g) * p.P + (slot_abs % p.P)) * D;
+      const size_t src = ((size_t)bi * p.Hkv + g) * D;
+      for (int e = threadIdx.x; e < D / 4; e += kThreads) {
+        // pairs (j, j + 1) of the first half with the same pairs of the second half, j = 2e
+        const uint32_t a = *reinterpret_cast<const uint32_t*>(p.k_new + src + 2 * e);
+        const uint32_t b = *reinterpret_cast<const uint32_t*>(p.k_new + src + D / 2 + 2 * e);
+        double cs[2], sn[2];
+        rope_sincos(tpos, p.inv_freq[2 * e], cs[0], sn[0]);
+        rope_sincos(tpos, p.inv_freq[2 * e + 1], cs[1], sn[1]);
+        uint32_t lo, hi;
+        rope_rotate2(a, b, cs, sn, lo, hi);
+        *reinterpret_cast<uint32_t*>(p.kpool + dst + 2 * e) = lo;
+        *reinterpret_cast<uint32_t*>(p.kpool + dst + D / 2 + 2 * e) = hi;
+      }
+      for (int e = threadIdx.x; e < D / 2; e += kThreads)
+        *reinterpret_cast<uint32_t*>(p.vpool + dst + 2 * e) =
+            *reinterpret_cast<const uint32_t*>(p.v_new + src + 2 * e);
+      fence_proxy_async_global();
+    }
+  }
   // q of the G heads: RoPE at the token's position (float64 rotation, one bf16
-  // rounding, as the cache keys), then scaled by log2(e)/sqrt(d).
-  const int tpos = p.pos[bi];
+  // rounding, as the cache keys), scaled by log2(e)/sqrt(d), stored per quarter
+  // with padding so that the four quarters' broadcasts fall in different banks.
   for (int e = threadIdx.x; e < G * (D / 2); e += kThreads) {
     const int h = e / (D / 2), j = e % (D / 2);
     const bf16* qr = p.q + ((size_t)bi * p.Hq + g * G + h) * D;
     const double x1 = __bfloat162float(qr[j]), x2 = __bfloat162float(qr[j + D / 2]);
     double cs, sn;
     rope_sincos(tpos, p.inv_freq[j], cs, sn);
-    qs[h * D + j] = __bfloat162float(__double2bfloat16(x1 * cs - x2 * sn)) * p.scale_log2;
-    qs[h * D + j + D / 2] = __bfloat162float(__double2bfloat16(x2 * cs + x1 * sn)) * p.scale_log2;
+    const int d1 = j, d2 = j + D / 2;
+    qs[(h * 4 + d1 / DQ) * QPAD + d1 % DQ] = __bfloat162float(__double2bfloat16(x1 * cs - x2 * sn)) * p.scale_log2;
+    qs[(h * 4 + d2 / DQ) * QPAD + d2 % DQ] = __bfloat162float(__double2bfloat16(x2 * cs + x1 * sn)) * p.scale_log2;
   }
   __syncthreads();
 
@@ -166,145 +189,163 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- compute
-    constexpr int DPT = D / 8;                  // QK: dims per thread (one eighth of d)
-    constexpr int DPL = D / 32;                 // PV: dims per lane
-    const int t = threadIdx.x;
-    const int kp = t & 31, e8 = t >> 5;         // QK: key pair, dim eighth (= warp)
-    float m_run = -INFINITY, l_run = 0.f;       // warp h < G: stats of head h
-    float acc[G][DPL];
+    const int kk = lane >> 2, qd = lane & 3;  // QK: key within the warp's 8, quarter of d
+    float* ps = ps_all + warp * 8 * G;         // this warp's P: [8 keys][G]
+    float m_run[G], l_run[G], acc[G][DPL];
 #pragma unroll
-    for (int h = 0; h < G; ++h)
+    for (int h = 0; h < G; ++h) {
+      m_run[h] = -INFINITY;
+      l_run[h] = 0.f;
 #pragma unroll
       for (int i = 0; i < DPL; ++i) acc[h][i] = 0.f;
+    }
     bool ok = true;
 
     for (int tt = 0; tt < ntiles; ++tt) {
       const int s = tt % NST;
-      const bool arrived = mbar_wait(&full[s], (tt / NST) & 1, kDevTimeoutSoftmax);
+      ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (tt / NST) & 1, kDevTimeoutSoftmax));
+      if (!ok) break;
       const uint8_t* kt = smem + s * S::kStage;
       const uint8_t* vt = kt + S::kTile;
+      const int key = 8 * warp + kk;
 
-      // 1. partial dot products over dims [DPT e8, DPT e8 + DPT) for keys kp, kp + 32
-      {
-        float d0[G], d1[G];
+      // QK over this lane's quarter, then across the key's four lanes.
+      float sc[G];
 #pragma unroll
-        for (int h = 0; h < G; ++h) d0[h] = d1[h] = 0.f;
+      for (int h = 0; h < G; ++h) sc[h] = 0.f;
 #pragma unroll
-        for (int ch = 0; ch < DPT / 8; ++ch) {
-          const int dbase = DPT * e8 + 8 * ch;
-          const uint4 ka = *reinterpret_cast<const uint4*>(kt + tile_off(kp, dbase));
-          const uint4 kb = *reinterpret_cast<const uint4*>(kt + tile_off(kp + 32, dbase));
-          const uint32_t* wa = reinterpret_cast<const uint32_t*>(&ka);
-          const uint32_t* wb = reinterpret_cast<const uint32_t*>(&kb);
+      for (int i = 0; i < DQ / 8; ++i) {
+        const uint4 kv = *reinterpret_cast<const uint4*>(kt + tile_off(key, qd * DQ + 8 * i));
+        const uint32_t* w = reinterpret_cast<const uint32_t*>(&kv);
+        float kf[8];
 #pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const float4 q0 = *reinterpret_cast<const float4*>(qs + h * D + dbase);
-            const float4 q1 = *reinterpret_cast<const float4*>(qs + h * D + dbase + 4);
-            const float qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float2 fa = unpack_bf16x2(wa[i]);
-              const float2 fb = unpack_bf16x2(wb[i]);
-              d0[h] = fmaf(qv[2 * i], fa.x, fmaf(qv[2 * i + 1], fa.y, d0[h]));
-              d1[h] = fmaf(qv[2 * i], fb.x, fmaf(qv[2 * i + 1], fb.y, d1[h]));
-            }
-          }
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = unpack_bf16x2(w[e]);
+          kf[2 * e] = f.x;
+          kf[2 * e + 1] = f.y;
         }
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          part[(e8 * G + h) * kTileKeys + kp] = d0[h];
-          part[(e8 * G + h) * kTileKeys + kp + 32] = d1[h];
+          const float* qrow = qs + (h * 4 + qd) * QPAD + 8 * i;
+          const float4 q0 = *reinterpret_cast<const float4*>(qrow);
+          const float4 q1 = *reinterpret_cast<const float4*>(qrow + 4);
+          float a = sc[h];
+          a = fmaf(q0.x, kf[0], a);
+          a = fmaf(q0.y, kf[1], a);
+          a = fmaf(q0.z, kf[2], a);
+          a = fmaf(q0.w, kf[3], a);
+          a = fmaf(q1.x, kf[4], a);
+          a = fmaf(q1.y, kf[5], a);
+          a = fmaf(q1.z, kf[6], a);
+          a = fmaf(q1.w, kf[7], a);
+          sc[h] = a;
         }
       }
-      ok = bar_compute_all(arrived);
-      if (!ok) break;
-
-      // 2. online softmax, warp h < G owns head h (keys lane and lane + 32)
-      if (warp < G) {
-        const int h = warp;
-        float s0 = 0.f, s1 = 0.f;
+      const bool valid = (k_begin + tt * kTileKeys + key) < k_end;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          s0 += part[(e * G + h) * kTileKeys + lane];
-          s1 += part[(e * G + h) * kTileKeys + lane + 32];
-        }
-        const int kg = k_begin + tt * kTileKeys;
-        if (kg + lane >= k_end) s0 = -INFINITY;
-        if (kg + lane + 32 >= k_end) s1 = -INFINITY;
-        float mt = fmaxf(s0, s1);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
-        const float m_new = fmaxf(m_run, mt);   // the tile's first key is always valid
-        const float alpha = ex2_approx(m_run - m_new);
-        const float p0 = ex2_approx(s0 - m_new), p1 = ex2_approx(s1 - m_new);
-        float ls = p0 + p1;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, off);
-        l_run = l_run * alpha + ls;
-        m_run = m_new;
-        ps[lane * G + h] = p0;
-        ps[(lane + 32) * G + h] = p1;
-        if (lane == 0) stat[h] = alpha;
+      for (int h = 0; h < G; ++h) {
+        sc[h] += __shfl_xor_sync(0xffffffffu, sc[h], 1);
+        sc[h] += __shfl_xor_sync(0xffffffffu, sc[h], 2);
+        if (!valid) sc[h] = -INFINITY;
       }
-      bar_compute();
-
-      // 3. P V: warp w takes keys [8w, 8w + 8); lane owns dims [DPL lane, DPL lane + DPL)
-      {
-        float al[G];
+      // Online softmax over the warp's 8 keys (lanes 4kk..4kk+3 hold key kk).
+      float al[G];
 #pragma unroll
-        for (int h = 0; h < G; ++h) al[h] = stat[h];
-#pragma unroll
-        for (int h = 0; h < G; ++h)
-#pragma unroll
-          for (int i = 0; i < DPL; ++i) acc[h][i] *= al[h];
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const int key = 8 * warp + kk;
-          float vf[DPL];
-          if constexpr (DPL == 4) {
-            const uint2 vv = *reinterpret_cast<const uint2*>(vt + tile_off(key, 4 * lane));
-            const float2 v01 = unpack_bf16x2(vv.x), v23 = unpack_bf16x2(vv.y);
-            vf[0] = v01.x; vf[1] = v01.y; vf[2] = v23.x; vf[3] = v23.y;
-          } else {
-            const float2 v01 = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(vt + tile_off(key, 2 * lane)));
-            vf[0] = v01.x; vf[1] = v01.y;
-          }
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const float pw = ps[key * G + h];
-#pragma unroll
-            for (int i = 0; i < DPL; ++i) acc[h][i] = fmaf(pw, vf[i], acc[h][i]);
-          }
-        }
+      for (int h = 0; h < G; ++h) {
+        float mt = sc[h];
+        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 4));
+        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 8));
+        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
+        const float m_new = fmaxf(m_run[h], mt);
+        const float mu = (m_new == -INFINITY) ? 0.f : m_new;
+        al[h] = ex2_approx(m_run[h] - mu);
+        const float pv = ex2_approx(sc[h] - mu);
+        float ls = pv;
+        ls += __shfl_xor_sync(0xffffffffu, ls, 4);
+        ls += __shfl_xor_sync(0xffffffffu, ls, 8);
+        ls += __shfl_xor_sync(0xffffffffu, ls, 16);
+        l_run[h] = l_run[h] * al[h] + ls;
+        m_run[h] = m_new;
+        if (qd == 0) ps[kk * G + h] = pv;
       }
-      bar_compute();
-      if (t == 0) mbar_arrive(&empty[s]);
-    }
-
-    // Final reduction over the 8 warps (reusing the stage buffers: all consumed).
-    if (ok) {
-      float* red = reinterpret_cast<float*>(smem);   // [8][G][D]
+      __syncwarp();
+      // P V: lane owns dims [DPL lane, DPL lane + DPL) of the G outputs.
 #pragma unroll
       for (int h = 0; h < G; ++h)
 #pragma unroll
-        for (int i = 0; i < DPL; ++i) red[(warp * G + h) * D + DPL * lane + i] = acc[h][i];
-      if (warp < G && lane == 0) {
-        stat[G + warp] = m_run;
-        stat[2 * G + warp] = l_run;
-      }
-      bar_compute();
-      const size_t rows = (size_t)p.B * p.Hq;
-      for (int idx = t; idx < G * D; idx += kCompute) {
-        const int h = idx / D;
-        float sum = 0.f;
+        for (int i = 0; i < DPL; ++i) acc[h][i] *= al[h];
 #pragma unroll
-        for (int w = 0; w < 8; ++w) sum += red[(w * G + h) * D + (idx % D)];
-        const float l = stat[2 * G + h];
-        const size_t row = (size_t)bi * p.Hq + g * G + h;
-        p.o_ws[((size_t)c * rows + row) * D + (idx % D)] = (l > 0.f) ? sum / l : 0.f;
-        if (idx % D == 0)
-          p.lse_ws[(size_t)c * rows + row] = (l > 0.f) ? (stat[G + h] + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+      for (int j = 0; j < 8; ++j) {
+        const int vkey = 8 * warp + j;
+        float vf[DPL];
+        if constexpr (DPL == 4) {
+          const uint2 vv = *reinterpret_cast<const uint2*>(vt + tile_off(vkey, 4 * lane));
+          const float2 v01 = unpack_bf16x2(vv.x), v23 = unpack_bf16x2(vv.y);
+          vf[0] = v01.x;
+          vf[1] = v01.y;
+          vf[2] = v23.x;
+          vf[3] = v23.y;
+        } else {
+          const float2 v01 = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(vt + tile_off(vkey, 2 * lane)));
+          vf[0] = v01.x;
+          vf[1] = v01.y;
+        }
+        float pj[G];
+        if constexpr (G % 4 == 0) {
+#pragma unroll
+          for (int h = 0; h < G; h += 4) {
+            const float4 p4 = *reinterpret_cast<const float4*>(ps + j * G + h);
+            pj[h] = p4.x;
+            pj[h + 1] = p4.y;
+            pj[h + 2] = p4.z;
+            pj[h + 3] = p4.w;
+          }
+        } else {
+#pragma unroll
+          for (int h = 0; h < G; ++h) pj[h] = ps[j * G + h];
+        }
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+#pragma unroll
+          for (int i = 0; i < DPL; ++i) acc[h][i] = fmaf(pj[h], vf[i], acc[h][i]);
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+
+    // Combine the 8 warps (reusing the stage buffers once every tile is consumed).
+    // A warp that gave up a wait still joins both barriers, so none is left waiting.
+    bar_compute();
+    float* red = reinterpret_cast<float*>(smem);  // [8][G][D] accumulators
+    float* st = red + 8 * G * D;                  // [8][G][2]: m, l
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) red[(warp * G + h) * D + DPL * lane + i] = acc[h][i];
+      if (lane == 0) {
+        st[(warp * G + h) * 2] = m_run[h];
+        st[(warp * G + h) * 2 + 1] = l_run[h];
+      }
+    }
+    bar_compute();
+    const size_t rows = (size_t)p.B * p.Hq;
+    for (int idx = threadIdx.x; idx < G * D; idx += kCompute) {
+      const int h = idx / D, dd = idx % D;
+      float mstar = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) mstar = fmaxf(mstar, st[(w * G + h) * 2]);
+      float sum = 0.f, l = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) {
+        const float mw = st[(w * G + h) * 2];
+        const float f = (mw == -INFINITY) ? 0.f : ex2_approx(mw - mstar);
+        sum += f * red[(w * G + h) * D + dd];
+        l += f * st[(w * G + h) * 2 + 1];
+      }
+      const size_t row = (size_t)bi * p.Hq + g * G + h;
+      p.o_ws[((size_t)c * rows + row) * D + dd] = (l > 0.f) ? sum / l : 0.f;
+      if (dd == 0)
+        p.lse_ws[(size_t)c * rows + row] = (l > 0.f) ? (mstar + __log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
   }
 }
@@ -348,10 +389,12 @@ cudaError_t launch_dg(const DecParams& p, const CUtensorMap& mk, const CUtensorM
 
 }  // namespace
 
+cudaError_t read_and_clear_error_decode(int* code) { return read_and_clear_tu_error(code); }
+
 int decode_num_chunks(int n_keys, int chunk) { return (n_keys + chunk - 1) / chunk; }
 
-// Chunks per (sequence, KV head) so that the grid is one wave of two CTAs per SM;
-// the chunk is a multiple of the 64-key tile.
+// Chunks per (sequence, KV head) so that the grid is one wave of kCtasPerSm CTAs
+// per SM; the chunk is a multiple of the 64-key tile.
 int decode_pick_chunk(int B, int Hkv, int G, int n_keys, int num_sms) {
   (void)G;
   long long per_head = (long long)kCtasPerSm * num_sms / ((long long)B * Hkv);
@@ -380,11 +423,13 @@ size_t decode_smem_bytes(int d, int G, int chunk) {
   }
 }
 
-cudaError_t read_and_clear_error_decode(int* code) { return read_and_clear_tu_error(code); }
-
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t st) {
   DecParams p;
   p.q = reinterpret_cast<const bf16*>(a.q);
+  p.k_new = reinterpret_cast<const bf16*>(a.k_new);
+  p.v_new = reinterpret_cast<const bf16*>(a.v_new);
+  p.kpool = reinterpret_cast<bf16*>(a.cache.k_pool);
+  p.vpool = reinterpret_cast<bf16*>(a.cache.v_pool);
   p.pos = a.pos;
   p.page_table = a.cache.page_table;
   p.o_ws = a.o_ws;

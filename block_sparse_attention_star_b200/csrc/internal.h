@@ -62,6 +62,8 @@ cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t st, const char** 
 struct DecodeLaunch {
   int B, Hq, Hkv, d;
   const void* q;          // [B][Hq][d] bf16 (pre-RoPE)
+  const void* k_new;      // [B][Hkv][d] bf16 (pre-RoPE): appended at slot n_keys - 1 by the kernel
+  const void* v_new;      // [B][Hkv][d] bf16
   const int32_t* pos;     // [B] position of the decoded token
   int n_keys;             // keys [0, n_keys) of every sequence
   int chunk;              // keys per CTA

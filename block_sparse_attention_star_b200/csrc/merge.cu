@@ -26,38 +26,53 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(int parts_per_group, lon
   const int group = blockIdx.y;
   if (row >= rows) return;
   const long long part0 = (long long)group * parts_per_group;
+  const int np = parts_per_group;
 
+  // LSE statistics: the lanes take the partials 32 at a time.
   float m = -INFINITY;
-  for (int i = 0; i < parts_per_group; ++i) {
-    const float li = lse_in[(part0 + i) * rows + row];
+  for (int i = lane; i < np; i += 32) {
+    const float li = __ldg(lse_in + (part0 + i) * rows + row);
     if (isfinite(li)) m = fmaxf(m, li);
   }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
   float acc[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
   float lse = -INFINITY;
   if (m != -INFINITY) {
     float s = 0.f;
-    for (int i = 0; i < parts_per_group; ++i) {
-      const float li = lse_in[(part0 + i) * rows + row];
+    for (int i = lane; i < np; i += 32) {
+      const float li = __ldg(lse_in + (part0 + i) * rows + row);
       if (isfinite(li)) s += expf(li - m);
     }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
     lse = m + logf(s);
-    for (int i = 0; i < parts_per_group; ++i) {
-      const float li = lse_in[(part0 + i) * rows + row];
-      if (!isfinite(li)) continue;
-      const float w = expf(li - lse);
-      const float* src = o_in + ((part0 + i) * rows + row) * D + lane * PER;
-      if constexpr (PER == 4) {
-        const float4 v = __ldg(reinterpret_cast<const float4*>(src));
-        acc[0] += w * v.x;
-        acc[1] += w * v.y;
-        acc[2] += w * v.z;
-        acc[3] += w * v.w;
-      } else {
-        const float2 v = __ldg(reinterpret_cast<const float2*>(src));
-        acc[0] += w * v.x;
-        acc[1] += w * v.y;
+    // O: each lane owns PER consecutive columns; weights are broadcast from the lane
+    // that computed them, and the loads of several partials are in flight at once.
+    for (int base = 0; base < np; base += 32) {
+      float w = 0.f;
+      if (base + lane < np) {
+        const float li = __ldg(lse_in + (part0 + base + lane) * rows + row);
+        if (isfinite(li)) w = expf(li - lse);
+      }
+      const int cnt = min(32, np - base);
+#pragma unroll 4
+      for (int j = 0; j < cnt; ++j) {
+        const float wj = __shfl_sync(0xffffffffu, w, j);
+        const float* src = o_in + ((part0 + base + j) * rows + row) * D + lane * PER;
+        if constexpr (PER == 4) {
+          const float4 v = __ldg(reinterpret_cast<const float4*>(src));
+          acc[0] = fmaf(wj, v.x, acc[0]);
+          acc[1] = fmaf(wj, v.y, acc[1]);
+          acc[2] = fmaf(wj, v.z, acc[2]);
+          acc[3] = fmaf(wj, v.w, acc[3]);
+        } else {
+          const float2 v = __ldg(reinterpret_cast<const float2*>(src));
+          acc[0] = fmaf(wj, v.x, acc[0]);
+          acc[1] = fmaf(wj, v.y, acc[1]);
+        }
       }
     }
   }

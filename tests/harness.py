@@ -85,9 +85,29 @@ def err(gpu, ref) -> Err:
     return Err(float(d.max()) if d.size else 0.0, float(d.mean()) if d.size else 0.0)
 
 
+def bf16_spacing(x) -> np.ndarray:
+    """Distance between adjacent bf16 values at |x| (8 significant bits)."""
+    m = np.maximum(np.abs(np.asarray(x, dtype=np.float64)), 2.0 ** -126)
+    return np.ldexp(1.0, np.floor(np.log2(m)).astype(np.int64) - 7)
+
+
 def assert_out(gpu, ref, what: str):
+    """bf16 outputs against the float64 oracle.
+
+    Mean abs <= 2e-3 everywhere; max abs <= 1.5e-2 wherever the bf16 output
+    format can represent it, i.e. |O| < 4.  From |O| = 4 up, rounding an exact
+    result to bf16 alone can be off by half the spacing (0.0156 at [4, 8)), so
+    there the per-element bound is half the spacing plus 4e-3.
+    """
     e = err(gpu, ref)
-    assert e.ok(), f"{what}: max abs {e.max_abs:.3e} (<= {MAX_ABS}), mean abs {e.mean_abs:.3e} (<= {MEAN_ABS})"
+    g = to64(gpu) if isinstance(gpu, torch.Tensor) else np.asarray(gpu, dtype=np.float64)
+    r = np.asarray(ref, dtype=np.float64)
+    bound = np.maximum(MAX_ABS, 0.5 * bf16_spacing(r) + 4e-3)
+    over = np.abs(g - r) > bound
+    worst = np.unravel_index(np.argmax(np.abs(g - r) - bound), r.shape) if r.size else None
+    assert not over.any() and e.mean_abs <= MEAN_ABS, (
+        f"{what}: max abs {e.max_abs:.3e}, mean abs {e.mean_abs:.3e} (<= {MEAN_ABS}); "
+        f"{int(over.sum())} elements over the bound, worst at {worst}: gpu {g[worst]:.6f} oracle {r[worst]:.6f}")
     return e
 
 
