@@ -1,31 +1,41 @@
-// Star Attention decode: one generated token attends to the whole cache
-// ("Star Attention: Efficient LLM Inference over Long Sequences", abstract:
+// Star Attention decode: one generated token per sequence attends to the whole
+// cache ("Star Attention: Efficient LLM Inference over Long Sequences", abstract:
 // response tokens attend to all prior cached tokens; "Star Attention 完全拆解(一)",
 // "Phase 2: 局部注意力与本地统计量": each block yields a local output and its
 // softmax statistic, merged exactly in "组装全局结果").
 //
-// HBM-bound: a step reads every cached K and V byte once.  The cache is cut into
-// chunks (a finer partition than blocks; the merge is associative, so chunk
-// partials merge to the same result as per-block partials).  One CTA per
-// (chunk, KV head, sequence) serves all G query heads of the group, so each K/V
-// byte is fetched once for G heads.  The grid is one wave of kCtasPerSm CTAs per SM.
+// HBM-bound: a step reads every cached K and V byte once.  The cache of each
+// (sequence, KV head) is cut into chunks of whole 128-key tiles (a finer partition
+// than blocks; the merge is associative, so chunk partials merge to the same result
+// as per-block partials).  A work item is one (sequence, KV head, chunk); a
+// persistent CTA per SM takes items round-robin and streams their tiles through
+// one TMA ring, so the loads never stop at item boundaries.
 //
-// The CTA that owns the last chunk of a (sequence, KV head) first appends the new
-// token: RoPE(k) (float64 rotation, one bf16 rounding, like star_kv_append) and v
-// go to cache slot n_keys - 1, made visible to its own TMA loads by a proxy fence.
+// The G query heads of a GQA group against one 128-key tile are a dense product
+// (G x d times d x 128).  It runs on the tensor core in transposed form, so that
+// the 128 keys fill the UMMA M dimension and the heads, padded to 16, are N:
+//   S^T [128 keys x 16]  = K_tile [128 x d] . Q_g^T             (K-major A and B)
+//   O^T [d x 16]         = V_tile^T [d x 128 keys] . P^T        (MN-major A, K-major B)
+// K and V tiles land by TMA in the Phase-1 layout ([key][64 d] boxes, 128-byte
+// swizzle), which is exactly the K-major A operand of S^T and the MN-major A
+// operand of O^T.  Each tile's O^T goes to a fresh TMEM accumulator and is added
+// into registers with the online-softmax rescale, so no TMEM value is rewritten.
 //
-// CTA: warp 8 is the TMA producer (64-key K and V tiles, 128-byte swizzle, an
-// NST-stage ring, no multicast); warps 0-7 compute.  Warp w owns keys
-// [8w, 8w + 8) of every tile and keeps its own online softmax (running max m and
-// sum l per head, base 2), so there is no CTA barrier per tile:
-//   QK: lane = (key kk = lane / 4, quarter = lane % 4); it dots its quarter of
-//       the key with the same quarter of the G query vectors (shared-memory
-//       broadcast from a padded layout); two shuffles finish the dot products.
-//   softmax: max and sum over the warp's 8 keys by shuffles; P goes to a small
-//       per-warp shared buffer.
-//   PV: lane owns d/32 dims of the G outputs and accumulates the 8 keys.
-// At the end the 8 warps' (m, l, O) are combined and the chunk's normalised O and
-// natural-log LSE are written for the merge kernel.
+// Softmax threads own one key of S^T and one dimension of O^T each (TMEM lane =
+// thread), so a tile costs them a few dozen instructions: the kernel streams at
+// HBM rate instead of being bound by instruction issue, as a CUDA-core dot-product
+// formulation of the same step is (about 80 instructions per key and head group).
+//
+// Before any load, the CTA owning the last chunk of a (sequence, KV head) appends
+// the new token: RoPE(k) (float64 rotation, one bf16 rounding, like
+// star_kv_append) and v go to cache slot n_keys - 1, made visible to its own TMA
+// loads by a proxy fence.
+//
+// CTA (256 threads, one per SM):
+//   warp 0     TMA producer (K and V rings, no multicast)
+//   warp 1     TMEM allocation and MMA issuer
+//   warps 2-3  prologue only (appends, q)
+//   warps 4-7  softmax and O accumulation: thread = TMEM lane 32 (w - 4) + lane
 #include "common.cuh"
 #include "internal.h"
 
@@ -34,12 +44,13 @@
 namespace star {
 namespace {
 
-constexpr int kCompute = 256;            // compute threads (8 warps)
-constexpr int kThreads = kCompute + 32;  // + producer warp
-constexpr int kTileKeys = 64;
-constexpr int kMaxChunk = 1 << 16;
-constexpr int kCtasPerSm = 2;
-constexpr int kStages = 3;
+constexpr int kThreads = 256;
+constexpr int kTileKeys = 128;           // UMMA M of S^T, K of O^T
+constexpr int kStages = 3;               // K/V ring depth
+constexpr int kMaxItems = 8;             // items per CTA per launch (q of each stays in shared memory)
+constexpr uint32_t kTmemCols = 64;       // S^T: [0,16) [16,32); O^T: [32,48) [48,64)
+constexpr uint32_t kIdescQK = umma_idesc_bf16(128, 16, 0, 0);
+constexpr uint32_t kIdescPV = umma_idesc_bf16(128, 16, 1, 0);
 
 struct DecParams {
   const bf16* q;       // [B][Hq][D]
@@ -49,304 +60,426 @@ struct DecParams {
   bf16* vpool;
   const int32_t* pos;  // [B]
   const int32_t* page_table;
-  float* o_ws;
-  float* lse_ws;
+  float* o_ws;         // [nchunks][B*Hq][D]
+  float* lse_ws;       // [nchunks][B*Hq]
   int max_pages, num_pages, P;
   int B, Hq, Hkv, n_keys, chunk, nchunks;
+  int item_base, num_items;  // this launch: items [item_base, num_items)
   float scale_log2;
   double inv_freq[kMaxHalfDim];
 };
 
-template <int D, int G>
+template <int D>
 struct DecSmem {
-  static constexpr int NST = kStages;
-  static constexpr int QPAD = D / 4 + 4;                  // floats per (head, quarter) row
-  static constexpr int kTile = kTileKeys * D * 2;         // one K or V tile
-  static constexpr int kStage = 2 * kTile;                // K then V
-  static constexpr int kQ = NST * kStage;                 // f32 [G][4][QPAD]
-  static constexpr int kP = kQ + G * 4 * QPAD * 4;        // f32 [8 warps][8 keys][G]
-  static constexpr int kBar = (kP + 8 * 8 * G * 4 + 7) / 8 * 8;
-  static constexpr int kEnd = kBar + 2 * NST * 8;
-  static constexpr int kBytes = kEnd + 1024;
-  static_assert(8 * G * (D + 2) * 4 <= NST * kStage, "final combine must fit in the stage buffers");
+  static constexpr int kTile = kTileKeys * D * 2;    // D/64 boxes of [128 keys][128 B]
+  // The V ring comes first: for D = 64 the M = 128 view of a V tile reads the
+  // 16 KB after it (rows 64-127 of O^T, never used), which must be shared memory.
+  static constexpr int kV = 0;
+  static constexpr int kK = kV + kStages * kTile;
+  static constexpr int kQItem = (D / 64) * 1024;      // D/64 atoms of [8 heads][128 B]
+  static constexpr int kQ = kK + kStages * kTile;
+  static constexpr int kP = kQ + kMaxItems * kQItem;   // 2 buffers x 2 atoms (keys 0-63, 64-127)
+  static constexpr int kPad = kP + 2 * 2048;          // read by the N = 16 view of the last P atom
+  static constexpr int kXch = kPad + 1024;            // f32 [2][4 warps][8 heads]: warp maxima
+  static constexpr int kRed = kXch + 2 * 4 * 8 * 4;   // f32 [4 warps][8 heads][2]: sums
+  static constexpr int kBar = kRed + 4 * 8 * 2 * 4;
+  static constexpr int kNumBars = 4 * kStages + 6 * 2 + 2;
+  static constexpr int kSlot = kBar + kNumBars * 8;
+  static constexpr int kBytes = kSlot + 16 + 1024;    // + alignment slack
+  static_assert(kBytes <= 227 * 1024, "decode shared memory");
 };
 
-// Byte offset of element (key, d) in a swizzled 64-key tile: 64-element d halves
-// are separate [64 keys][128 B] boxes; 16-byte chunks are XOR-permuted by key % 8.
-__device__ __forceinline__ int tile_off(int key, int d) {
-  const int half = d >> 6, e = d & 63;
-  return half * (kTileKeys * 128) + key * 128 + ((((e >> 3) ^ (key & 7)) << 4) | ((e & 7) << 1));
+struct DecItem {
+  int bi, g, c, k_begin, k_end, ntiles;
+};
+
+__device__ __forceinline__ DecItem dec_item(const DecParams& p, int idx) {
+  DecItem it;
+  it.c = idx % p.nchunks;
+  it.g = (idx / p.nchunks) % p.Hkv;
+  it.bi = idx / (p.nchunks * p.Hkv);
+  it.k_begin = it.c * p.chunk;
+  it.k_end = min(it.k_begin + p.chunk, p.n_keys);
+  it.ntiles = (it.k_end - it.k_begin + kTileKeys - 1) / kTileKeys;
+  return it;
 }
 
-__device__ __forceinline__ void bar_compute() { asm volatile("bar.sync 1, %0;" ::"n"(kCompute) : "memory"); }
+// Byte offset of (row, element e) in a K-major 128-byte-swizzle atom of 8 rows x 64 bf16.
+__device__ __forceinline__ int sw128(int row, int e) {
+  return row * 128 + ((((e >> 3) ^ (row & 7)) << 4) | ((e & 7) << 1));
+}
+
+// tcgen05.ld, 32 lanes x N columns of 32 bit (N = 1, 2, 4, 8).
+template <int N>
+__device__ __forceinline__ void tmem_ld_n(uint32_t taddr, uint32_t (&r)[N]);
+template <>
+__device__ __forceinline__ void tmem_ld_n<1>(uint32_t taddr, uint32_t (&r)[1]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r[0]) : "r"(taddr));
+}
+template <>
+__device__ __forceinline__ void tmem_ld_n<2>(uint32_t taddr, uint32_t (&r)[2]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(taddr));
+}
+template <>
+__device__ __forceinline__ void tmem_ld_n<4>(uint32_t taddr, uint32_t (&r)[4]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr));
+}
+template <>
+__device__ __forceinline__ void tmem_ld_n<8>(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+
+__device__ __forceinline__ float warp_max(float x) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(x));
+  return r;
+}
 
 __device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 
 template <int D, int G>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+__global__ void __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const __grid_constant__ DecParams p) {
-  using S = DecSmem<D, G>;
-  constexpr int NST = S::NST;
-  constexpr int QPAD = S::QPAD;
-  constexpr int DQ = D / 4;    // dims per quarter (QK)
-  constexpr int DPL = D / 32;  // dims per lane (PV)
+  using S = DecSmem<D>;
+  constexpr int NST = kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* qs = reinterpret_cast<float*>(smem + S::kQ);
-  float* ps_all = reinterpret_cast<float*>(smem + S::kP);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBar);
-  uint64_t* empty = full + NST;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
+  uint64_t* k_full = bars;
+  uint64_t* k_empty = bars + NST;
+  uint64_t* v_full = bars + 2 * NST;
+  uint64_t* v_empty = bars + 3 * NST;
+  uint64_t* s_full = bars + 4 * NST;  // [2] each
+  uint64_t* s_empty = s_full + 2;
+  uint64_t* p_full = s_full + 4;
+  uint64_t* o_full = s_full + 6;
+  uint64_t* o_empty = s_full + 8;
+  uint64_t* x_bar = s_full + 10;
+  uint64_t* red_bar = s_full + 12;
+  uint64_t* drain = s_full + 13;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kSlot);
+  float* xch = reinterpret_cast<float*>(smem + S::kXch);
+  float* red = reinterpret_cast<float*>(smem + S::kRed);
 
-  const int c = blockIdx.x % p.nchunks;
-  const int g = (blockIdx.x / p.nchunks) % p.Hkv;
-  const int bi = blockIdx.x / (p.nchunks * p.Hkv);
-  const int k_begin = c * p.chunk;
-  const int k_end = min(k_begin + p.chunk, p.n_keys);
-  const int ntiles = (k_end - k_begin + kTileKeys - 1) / kTileKeys;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int tpos = p.pos[bi];
+  const int first = p.item_base + blockIdx.x;
+  const int n_my = min(kMaxItems, (p.num_items - first + (int)gridDim.x - 1) / (int)gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 8);
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&s_empty[b], 4);
+      mbar_init(&p_full[b], 4);
+      mbar_init(&o_full[b], 1);
+      mbar_init(&o_empty[b], 4);
+      mbar_init(&x_bar[b], 4);
+    }
+    mbar_init(red_bar, 4);
+    mbar_init(drain, 1);
     fence_barrier_init();
   }
-  // The owner of the last chunk appends the new token (head g) before any load.
-  if (c == p.nchunks - 1) {
-    const int slot_abs = p.n_keys - 1;
-    const int page = p.page_table[(size_t)bi * p.max_pages + slot_abs / p.P];
-    if (page < 0 || page >= p.num_pages) {
-      if (threadIdx.x == 0) record_error(kDevBadPage);
-    } else {
-      const size_t dst = (((size_t)page * p.Hkv + g) * p.P + (slot_abs % p.P)) * D;
-      const size_t src = ((size_t)bi * p.Hkv + g) * D;
-      for (int e = threadIdx.x; e < D / 4; e += kThreads) {
-        // pairs (j, j + 1) of the first half with the same pairs of the second half, j = 2e
-        const uint32_t a = *reinterpret_cast<const uint32_t*>(p.k_new + src + 2 * e);
-        const uint32_t b = *reinterpret_cast<const uint32_t*>(p.k_new + src + D / 2 + 2 * e);
-        double cs[2], sn[2];
-        rope_sincos(tpos, p.inv_freq[2 * e], cs[0], sn[0]);
-        rope_sincos(tpos, p.inv_freq[2 * e + 1], cs[1], sn[1]);
-        uint32_t lo, hi;
-        rope_rotate2(a, b, cs, sn, lo, hi);
-        *reinterpret_cast<uint32_t*>(p.kpool + dst + 2 * e) = lo;
-        *reinterpret_cast<uint32_t*>(p.kpool + dst + D / 2 + 2 * e) = hi;
-      }
-      for (int e = threadIdx.x; e < D / 2; e += kThreads)
-        *reinterpret_cast<uint32_t*>(p.vpool + dst + 2 * e) =
-            *reinterpret_cast<const uint32_t*>(p.v_new + src + 2 * e);
-      fence_proxy_async_global();
-    }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
   }
-  // q of the G heads: RoPE at the token's position (float64 rotation, one bf16
-  // rounding, as the cache keys), scaled by log2(e)/sqrt(d), stored per quarter
-  // with padding so that the four quarters' broadcasts fall in different banks.
-  for (int e = threadIdx.x; e < G * (D / 2); e += kThreads) {
-    const int h = e / (D / 2), j = e % (D / 2);
-    const bf16* qr = p.q + ((size_t)bi * p.Hq + g * G + h) * D;
-    const double x1 = __bfloat162float(qr[j]), x2 = __bfloat162float(qr[j + D / 2]);
-    double cs, sn;
-    rope_sincos(tpos, p.inv_freq[j], cs, sn);
-    const int d1 = j, d2 = j + D / 2;
-    qs[(h * 4 + d1 / DQ) * QPAD + d1 % DQ] = __bfloat162float(__double2bfloat16(x1 * cs - x2 * sn)) * p.scale_log2;
-    qs[(h * 4 + d2 / DQ) * QPAD + d2 % DQ] = __bfloat162float(__double2bfloat16(x2 * cs + x1 * sn)) * p.scale_log2;
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
   }
+  // q and P operands: the padding rows (heads G..15) are zeros.
+  for (int i = threadIdx.x; i < (S::kXch - S::kQ) / 16; i += kThreads)
+    reinterpret_cast<uint4*>(smem + S::kQ)[i] = make_uint4(0u, 0u, 0u, 0u);
   __syncthreads();
 
-  if (warp == 8) {
+  for (int ii = 0; ii < n_my; ++ii) {
+    const DecItem it = dec_item(p, first + ii * gridDim.x);
+    const int tpos = p.pos[it.bi];
+    // Append the new token (head g) when this item holds the cache's last key.
+    if (it.c == p.nchunks - 1) {
+      const int slot_abs = p.n_keys - 1;
+      const int page = p.page_table[(size_t)it.bi * p.max_pages + slot_abs / p.P];
+      if (page < 0 || page >= p.num_pages) {
+        if (threadIdx.x == 0) record_error(kDevBadPage);
+      } else {
+        const size_t dst = (((size_t)page * p.Hkv + it.g) * p.P + (slot_abs % p.P)) * D;
+        const size_t src = ((size_t)it.bi * p.Hkv + it.g) * D;
+        for (int e = threadIdx.x; e < D / 4; e += kThreads) {
+          // pairs (j, j + 1) of the first half with the same pairs of the second half, j = 2e
+          const uint32_t a = *reinterpret_cast<const uint32_t*>(p.k_new + src + 2 * e);
+          const uint32_t b = *reinterpret_cast<const uint32_t*>(p.k_new + src + D / 2 + 2 * e);
+          double cs[2], sn[2];
+          rope_sincos(tpos, p.inv_freq[2 * e], cs[0], sn[0]);
+          rope_sincos(tpos, p.inv_freq[2 * e + 1], cs[1], sn[1]);
+          uint32_t lo, hi;
+          rope_rotate2(a, b, cs, sn, lo, hi);
+          *reinterpret_cast<uint32_t*>(p.kpool + dst + 2 * e) = lo;
+          *reinterpret_cast<uint32_t*>(p.kpool + dst + D / 2 + 2 * e) = hi;
+        }
+        for (int e = threadIdx.x; e < D / 2; e += kThreads)
+          *reinterpret_cast<uint32_t*>(p.vpool + dst + 2 * e) =
+              *reinterpret_cast<const uint32_t*>(p.v_new + src + 2 * e);
+        fence_proxy_async_global();
+      }
+    }
+    // q of the G heads: RoPE at the token's position (float64 rotation, one bf16
+    // rounding, as the cache keys), as the K-major B operand [head][d].
+    uint8_t* qs = smem + S::kQ + ii * S::kQItem;
+    for (int e = threadIdx.x; e < G * (D / 2); e += kThreads) {
+      const int h = e / (D / 2), j = e % (D / 2);
+      const bf16* qr = p.q + ((size_t)it.bi * p.Hq + it.g * G + h) * D;
+      const double x1 = __bfloat162float(qr[j]), x2 = __bfloat162float(qr[j + D / 2]);
+      double cs, sn;
+      rope_sincos(tpos, p.inv_freq[j], cs, sn);
+      const int d1 = j, d2 = j + D / 2;
+      *reinterpret_cast<bf16*>(qs + (d1 / 64) * 1024 + sw128(h, d1 % 64)) = __double2bfloat16(x1 * cs - x2 * sn);
+      *reinterpret_cast<bf16*>(qs + (d2 / 64) * 1024 + sw128(h, d2 % 64)) = __double2bfloat16(x2 * cs + x1 * sn);
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  if (warp == 0) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
+      uint32_t kc = 0;
       bool ok = true;
-      for (int t = 0; t < ntiles && ok; ++t) {
-        const int s = t % NST;
-        ok = mbar_wait(&empty[s], ((t / NST) & 1) ^ 1, kDevTimeoutProducer);
-        if (!ok) break;
-        const int k0 = k_begin + t * kTileKeys;
-        int page = p.page_table[(size_t)bi * p.max_pages + k0 / p.P];
-        if (page < 0 || page >= p.num_pages) {
-          record_error(kDevBadPage);
-          page = 0;
-        }
-        const int slot = k0 % p.P;
-        mbar_arrive_expect_tx(&full[s], 2 * S::kTile);
-        uint8_t* dk = smem + s * S::kStage;
-        uint8_t* dv = dk + S::kTile;
+      for (int ii = 0; ii < n_my && ok; ++ii) {
+        const DecItem it = dec_item(p, first + ii * gridDim.x);
+        for (int t = 0; t < it.ntiles && ok; ++t, ++kc) {
+          const int k0 = it.k_begin + t * kTileKeys;
+          int page = p.page_table[(size_t)it.bi * p.max_pages + k0 / p.P];
+          if (page < 0 || page >= p.num_pages) {
+            record_error(kDevBadPage);
+            page = 0;
+          }
+          const int slot = k0 % p.P;
+          const int s = kc % NST;
+          const uint32_t ph = ((kc / NST) & 1) ^ 1;
+          ok = mbar_wait(&k_empty[s], ph, kDevTimeoutProducer);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&k_full[s], S::kTile);
 #pragma unroll
-        for (int h = 0; h < D / 64; ++h) {
-          tma_load_4d(dk + h * (kTileKeys * 128), &tmK, &full[s], h * 64, slot, g, page);
-          tma_load_4d(dv + h * (kTileKeys * 128), &tmV, &full[s], h * 64, slot, g, page);
+          for (int h = 0; h < D / 64; ++h)
+            tma_load_4d(smem + S::kK + s * S::kTile + h * (kTileKeys * 128), &tmK, &k_full[s], h * 64, slot, it.g,
+                        page);
+          ok = mbar_wait(&v_empty[s], ph, kDevTimeoutProducer);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&v_full[s], S::kTile);
+#pragma unroll
+          for (int h = 0; h < D / 64; ++h)
+            tma_load_4d(smem + S::kV + s * S::kTile + h * (kTileKeys * 128), &tmV, &v_full[s], h * 64, slot, it.g,
+                        page);
         }
       }
       // Every load issued has landed before the CTA may exit.
-      for (int s = 0; s < NST && s < ntiles; ++s) {
-        const int last = ntiles - 1 - ((ntiles - 1 - s) % NST);
-        mbar_wait(&full[s], (last / NST) & 1, kDevTimeoutProducer);
+      for (uint32_t s = 0; s < (uint32_t)NST && s < kc; ++s) {
+        const uint32_t last = kc - 1 - ((kc - 1 - s) % NST);
+        mbar_wait(&k_full[s], (last / NST) & 1, kDevTimeoutProducer);
+        mbar_wait(&v_full[s], (last / NST) & 1, kDevTimeoutProducer);
       }
     }
-    __syncwarp();
-  } else {
-    // ---------------------------------------------------------------- compute
-    const int kk = lane >> 2, qd = lane & 3;  // QK: key within the warp's 8, quarter of d
-    float* ps = ps_all + warp * 8 * G;         // this warp's P: [8 keys][G]
-    float m_run[G], l_run[G], acc[G][DPL];
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t sK = smem_u32(smem + S::kK), sV = smem_u32(smem + S::kV);
+      const uint32_t sQ = smem_u32(smem + S::kQ), sP = smem_u32(smem + S::kP);
+      bool issued = false;
+      // O^T_t = V_t^T P_t^T: V MN-major (d atoms 16 KB apart, 8-key groups 1 KB apart,
+      // 16 keys = 2 KB per K step); P K-major (64-key atoms 1 KB apart).
+      auto issue_pv = [&](uint32_t t) -> bool {
+        const int s = t % NST, b = t & 1;
+        if (!mbar_wait(&v_full[s], (t / NST) & 1, kDevTimeoutMma)) return false;
+        if (!mbar_wait(&p_full[b], (t >> 1) & 1, kDevTimeoutMma)) return false;
+        if (t >= 2 && !mbar_wait(&o_empty[b], ((t >> 1) & 1) ^ 1, kDevTimeoutMma)) return false;
+        tc_fence_after();
+        const uint32_t va = sV + s * S::kTile, pb = sP + b * 2048;
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      m_run[h] = -INFINITY;
-      l_run[h] = 0.f;
+        for (int kk = 0; kk < kTileKeys / 16; ++kk)
+          mma_ss(tbase + 32 + 16 * b, umma_desc_sw128(va + kk * 2048, kTileKeys * 128, 1024),
+                 umma_desc_sw128(pb + (kk / 4) * 1024 + (kk % 4) * 32, 16, 1024), kIdescPV, kk > 0 ? 1u : 0u);
+        mma_commit(&o_full[b]);
+        mma_commit(&v_empty[s]);
+        return true;
+      };
+      uint32_t j = 0;
+      bool ok = true;
+      for (int ii = 0; ii < n_my && ok; ++ii) {
+        const DecItem it = dec_item(p, first + ii * gridDim.x);
+        const uint32_t qa = sQ + ii * S::kQItem;
+        for (int t = 0; t < it.ntiles; ++t, ++j) {
+          const int s = j % NST, b = j & 1;
+          ok = mbar_wait(&k_full[s], (j / NST) & 1, kDevTimeoutMma);
+          if (ok && j >= 2) ok = mbar_wait(&s_empty[b], ((j >> 1) & 1) ^ 1, kDevTimeoutMma);
+          if (!ok) break;
+          tc_fence_after();
+          // S^T_j = K_j Q^T: K-major, 8-row groups 1 KB apart, 16-element K step = 32 B
+          // inside a 64-element atom; K atoms 16 KB apart, q atoms 1 KB apart.
+          const uint32_t ka = sK + s * S::kTile;
 #pragma unroll
-      for (int i = 0; i < DPL; ++i) acc[h][i] = 0.f;
-    }
-    bool ok = true;
-
-    for (int tt = 0; tt < ntiles; ++tt) {
-      const int s = tt % NST;
-      ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (tt / NST) & 1, kDevTimeoutSoftmax));
-      if (!ok) break;
-      const uint8_t* kt = smem + s * S::kStage;
-      const uint8_t* vt = kt + S::kTile;
-      const int key = 8 * warp + kk;
-
-      // QK over this lane's quarter, then across the key's four lanes.
-      float sc[G];
-#pragma unroll
-      for (int h = 0; h < G; ++h) sc[h] = 0.f;
-#pragma unroll
-      for (int i = 0; i < DQ / 8; ++i) {
-        const uint4 kv = *reinterpret_cast<const uint4*>(kt + tile_off(key, qd * DQ + 8 * i));
-        const uint32_t* w = reinterpret_cast<const uint32_t*>(&kv);
-        float kf[8];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = unpack_bf16x2(w[e]);
-          kf[2 * e] = f.x;
-          kf[2 * e + 1] = f.y;
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tbase + 16 * b, umma_desc_sw128(ka + (kk / 4) * (kTileKeys * 128) + (kk % 4) * 32, 16, 1024),
+                   umma_desc_sw128(qa + (kk / 4) * 1024 + (kk % 4) * 32, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+          issued = true;
+          mma_commit(&s_full[b]);
+          mma_commit(&k_empty[s]);
+          if (j >= 1) {
+            ok = issue_pv(j - 1);
+            if (!ok) break;
+          }
         }
+      }
+      if (ok && j >= 1) issue_pv(j - 1);
+      if (issued) {
+        // Every MMA this thread issued has completed before TMEM is released.
+        mma_commit(drain);
+        mbar_wait(drain, 0, kDevTimeoutMma);
+      }
+    }
+  } else if (warp >= 4) {
+    // ---------------------------------------------------------------- softmax + O
+    const int wi = warp - 4;
+    const uint32_t tl = tbase + ((uint32_t)(wi * 32) << 16);
+    const int kt = wi * 32 + lane;  // key of the tile (S^T lane) and dimension (O^T lane)
+    uint8_t* sP = smem + S::kP;
+    const size_t rows = (size_t)p.B * p.Hq;
+    uint32_t j = 0;
+    bool ok = true;
+    float o[G], al_prev[G];
+
+    // O_run = O_run * alpha_t + O^T_t for tile t (lane kt = dimension kt).
+    auto acc_o = [&](uint32_t t, const float (&al)[G]) -> bool {
+      const int b = t & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&o_full[b], (t >> 1) & 1, kDevTimeoutSoftmax))) return false;
+      tc_fence_after();
+      uint32_t r[G];
+      tmem_ld_n<G>(tl + 32 + 16 * b, r);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_empty[b]);
+#pragma unroll
+      for (int h = 0; h < G; ++h) o[h] = fmaf(o[h], al[h], __uint_as_float(r[h]));
+      return true;
+    };
+
+    for (int ii = 0; ii < n_my && ok; ++ii) {
+      const DecItem it = dec_item(p, first + ii * gridDim.x);
+      float m_run[G], lu[G], lr[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        m_run[h] = -INFINITY;
+        lu[h] = 0.f;
+        lr[h] = 0.f;
+        o[h] = 0.f;
+        al_prev[h] = 0.f;
+      }
+      for (int t = 0; t < it.ntiles; ++t, ++j) {
+        const int b = j & 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (j >> 1) & 1, kDevTimeoutSoftmax));
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t sr[G];
+        tmem_ld_n<G>(tl + 16 * b, sr);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[b]);
+        // Scores in base 2; keys past the chunk's end are masked.
+        const bool valid = it.k_begin + t * kTileKeys + kt < it.k_end;
+        float x[G];
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          const float* qrow = qs + (h * 4 + qd) * QPAD + 8 * i;
-          const float4 q0 = *reinterpret_cast<const float4*>(qrow);
-          const float4 q1 = *reinterpret_cast<const float4*>(qrow + 4);
-          float a = sc[h];
-          a = fmaf(q0.x, kf[0], a);
-          a = fmaf(q0.y, kf[1], a);
-          a = fmaf(q0.z, kf[2], a);
-          a = fmaf(q0.w, kf[3], a);
-          a = fmaf(q1.x, kf[4], a);
-          a = fmaf(q1.y, kf[5], a);
-          a = fmaf(q1.z, kf[6], a);
-          a = fmaf(q1.w, kf[7], a);
-          sc[h] = a;
+          x[h] = valid ? __uint_as_float(sr[h]) * p.scale_log2 : -INFINITY;
+          const float wm = warp_max(x[h]);
+          if (lane == 0) xch[(b * 4 + wi) * 8 + h] = wm;
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&x_bar[b]);
+        ok = __all_sync(0xffffffffu, mbar_wait(&x_bar[b], (j >> 1) & 1, kDevTimeoutSoftmax));
+        if (!ok) break;
+        // Tile max over the 4 warps; every tile has a valid key, so m_new is finite.
+        float al[G];
+        uint8_t* pt = sP + b * 2048 + (kt / 64) * 1024;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float* xw = xch + b * 32 + h;
+          const float tm = fmaxf(fmaxf(xw[0], xw[8]), fmaxf(xw[16], xw[24]));
+          const float m_new = fmaxf(m_run[h], tm);
+          al[h] = ex2_approx(m_run[h] - m_new);  // 0 on the first tile (m_run = -inf)
+          m_run[h] = m_new;
+          const float pv = ex2_approx(x[h] - m_new);
+          const bf16 pb = __float2bfloat16_rn(pv);
+          // lu: f32 sum for the log-sum-exp; lr: sum of the bf16 values the product uses.
+          lu[h] = fmaf(lu[h], al[h], pv);
+          lr[h] = fmaf(lr[h], al[h], __bfloat162float(pb));
+          *reinterpret_cast<bf16*>(pt + sw128(h, kt % 64)) = pb;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[b]);
+        if (t > 0) {
+          ok = acc_o(j - 1, al_prev);
+          if (!ok) break;
+        }
+#pragma unroll
+        for (int h = 0; h < G; ++h) al_prev[h] = al[h];
       }
-      const bool valid = (k_begin + tt * kTileKeys + key) < k_end;
+      if (!ok) break;
+      ok = acc_o(j - 1, al_prev);
+      if (!ok) break;
+      // Sums over the 128 keys of the tile lanes (thread partials), then the 4 warps.
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        sc[h] += __shfl_xor_sync(0xffffffffu, sc[h], 1);
-        sc[h] += __shfl_xor_sync(0xffffffffu, sc[h], 2);
-        if (!valid) sc[h] = -INFINITY;
+        float su = lu[h], sr = lr[h];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          su += __shfl_xor_sync(0xffffffffu, su, off);
+          sr += __shfl_xor_sync(0xffffffffu, sr, off);
+        }
+        if (lane == 0) {
+          red[(wi * 8 + h) * 2] = su;
+          red[(wi * 8 + h) * 2 + 1] = sr;
+        }
       }
-      // Online softmax over the warp's 8 keys (lanes 4kk..4kk+3 hold key kk).
-      float al[G];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(red_bar);
+      ok = __all_sync(0xffffffffu, mbar_wait(red_bar, ii & 1, kDevTimeoutSoftmax));
+      if (!ok) break;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        float mt = sc[h];
-        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 4));
-        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 8));
-        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
-        const float m_new = fmaxf(m_run[h], mt);
-        const float mu = (m_new == -INFINITY) ? 0.f : m_new;
-        al[h] = ex2_approx(m_run[h] - mu);
-        const float pv = ex2_approx(sc[h] - mu);
-        float ls = pv;
-        ls += __shfl_xor_sync(0xffffffffu, ls, 4);
-        ls += __shfl_xor_sync(0xffffffffu, ls, 8);
-        ls += __shfl_xor_sync(0xffffffffu, ls, 16);
-        l_run[h] = l_run[h] * al[h] + ls;
-        m_run[h] = m_new;
-        if (qd == 0) ps[kk * G + h] = pv;
-      }
-      __syncwarp();
-      // P V: lane owns dims [DPL lane, DPL lane + DPL) of the G outputs.
+        float Lu = 0.f, Lr = 0.f;
 #pragma unroll
-      for (int h = 0; h < G; ++h)
-#pragma unroll
-        for (int i = 0; i < DPL; ++i) acc[h][i] *= al[h];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int vkey = 8 * warp + j;
-        float vf[DPL];
-        if constexpr (DPL == 4) {
-          const uint2 vv = *reinterpret_cast<const uint2*>(vt + tile_off(vkey, 4 * lane));
-          const float2 v01 = unpack_bf16x2(vv.x), v23 = unpack_bf16x2(vv.y);
-          vf[0] = v01.x;
-          vf[1] = v01.y;
-          vf[2] = v23.x;
-          vf[3] = v23.y;
-        } else {
-          const float2 v01 = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(vt + tile_off(vkey, 2 * lane)));
-          vf[0] = v01.x;
-          vf[1] = v01.y;
+        for (int w = 0; w < 4; ++w) {
+          Lu += red[(w * 8 + h) * 2];
+          Lr += red[(w * 8 + h) * 2 + 1];
         }
-        float pj[G];
-        if constexpr (G % 4 == 0) {
-#pragma unroll
-          for (int h = 0; h < G; h += 4) {
-            const float4 p4 = *reinterpret_cast<const float4*>(ps + j * G + h);
-            pj[h] = p4.x;
-            pj[h + 1] = p4.y;
-            pj[h + 2] = p4.z;
-            pj[h + 3] = p4.w;
-          }
-        } else {
-#pragma unroll
-          for (int h = 0; h < G; ++h) pj[h] = ps[j * G + h];
-        }
-#pragma unroll
-        for (int h = 0; h < G; ++h)
-#pragma unroll
-          for (int i = 0; i < DPL; ++i) acc[h][i] = fmaf(pj[h], vf[i], acc[h][i]);
+        const size_t row = (size_t)it.bi * p.Hq + it.g * G + h;
+        if (kt < D) p.o_ws[((size_t)it.c * rows + row) * D + kt] = o[h] / Lr;
+        if (kt == h) p.lse_ws[(size_t)it.c * rows + row] = (m_run[h] + __log2f(Lu)) * 0.69314718055994531f;
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
     }
+  }
 
-    // Combine the 8 warps (reusing the stage buffers once every tile is consumed).
-    // A warp that gave up a wait still joins both barriers, so none is left waiting.
-    bar_compute();
-    float* red = reinterpret_cast<float*>(smem);  // [8][G][D] accumulators
-    float* st = red + 8 * G * D;                  // [8][G][2]: m, l
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-#pragma unroll
-      for (int i = 0; i < DPL; ++i) red[(warp * G + h) * D + DPL * lane + i] = acc[h][i];
-      if (lane == 0) {
-        st[(warp * G + h) * 2] = m_run[h];
-        st[(warp * G + h) * 2 + 1] = l_run[h];
-      }
-    }
-    bar_compute();
-    const size_t rows = (size_t)p.B * p.Hq;
-    for (int idx = threadIdx.x; idx < G * D; idx += kCompute) {
-      const int h = idx / D, dd = idx % D;
-      float mstar = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < 8; ++w) mstar = fmaxf(mstar, st[(w * G + h) * 2]);
-      float sum = 0.f, l = 0.f;
-#pragma unroll
-      for (int w = 0; w < 8; ++w) {
-        const float mw = st[(w * G + h) * 2];
-        const float f = (mw == -INFINITY) ? 0.f : ex2_approx(mw - mstar);
-        sum += f * red[(w * G + h) * D + dd];
-        l += f * st[(w * G + h) * 2 + 1];
-      }
-      const size_t row = (size_t)bi * p.Hq + g * G + h;
-      p.o_ws[((size_t)c * rows + row) * D + dd] = (l > 0.f) ? sum / l : 0.f;
-      if (dd == 0)
-        p.lse_ws[(size_t)c * rows + row] = (l > 0.f) ? (mstar + __log2f(l)) * 0.69314718055994531f : -INFINITY;
-    }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, kTmemCols);
   }
 }
 
@@ -373,9 +506,20 @@ bool make_tile_map(CUtensorMap* map, void* pool, int d, int P, int Hkv, int num_
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+int num_sms_cached() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
 template <int D, int G>
-cudaError_t launch_dg(const DecParams& p, const CUtensorMap& mk, const CUtensorMap& mv, cudaStream_t st) {
-  using S = DecSmem<D, G>;
+cudaError_t launch_dg(DecParams p, const CUtensorMap& mk, const CUtensorMap& mv, int total_items, cudaStream_t st) {
+  using S = DecSmem<D>;
   auto kern = decode_kernel<D, G>;
   static bool attr = false;
   if (!attr) {
@@ -383,8 +527,16 @@ cudaError_t launch_dg(const DecParams& p, const CUtensorMap& mk, const CUtensorM
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  kern<<<p.nchunks * p.Hkv * p.B, kThreads, S::kBytes, st>>>(mk, mv, p);
-  return cudaGetLastError();
+  const int grid = std::min(total_items, num_sms_cached());
+  // Each launch covers at most kMaxItems items per CTA.
+  for (int base = 0; base < total_items; base += grid * kMaxItems) {
+    p.item_base = base;
+    p.num_items = std::min(total_items, base + grid * kMaxItems);
+    kern<<<std::min(grid, p.num_items - base), kThreads, S::kBytes, st>>>(mk, mv, p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace
@@ -393,34 +545,34 @@ cudaError_t read_and_clear_error_decode(int* code) { return read_and_clear_tu_er
 
 int decode_num_chunks(int n_keys, int chunk) { return (n_keys + chunk - 1) / chunk; }
 
-// Chunks per (sequence, KV head) so that the grid is one wave of kCtasPerSm CTAs
-// per SM; the chunk is a multiple of the 64-key tile.
+// Keys per chunk (a multiple of the 128-key tile) for caches of up to n_keys keys:
+// the chunk count that minimises the tiles of the busiest CTA, counting each item
+// a quarter tile of overhead.
 int decode_pick_chunk(int B, int Hkv, int G, int n_keys, int num_sms) {
   (void)G;
-  long long per_head = (long long)kCtasPerSm * num_sms / ((long long)B * Hkv);
-  if (per_head < 1) per_head = 1;
-  long long chunk = (n_keys + per_head - 1) / per_head;
-  chunk = (chunk + kTileKeys - 1) / kTileKeys * kTileKeys;
-  chunk = std::max<long long>(kTileKeys, std::min<long long>(kMaxChunk, chunk));
-  return (int)chunk;
+  const long long tiles = std::max(1, (n_keys + kTileKeys - 1) / kTileKeys);
+  const long long bh = (long long)B * Hkv;
+  long long best_ct = tiles, best_cost = -1;
+  const long long nc_max = std::min<long long>(tiles, std::max<long long>(1, (long long)kMaxItems * num_sms / bh));
+  for (long long nc = 1; nc <= nc_max; ++nc) {
+    const long long ct = (tiles + nc - 1) / nc;
+    const long long nce = (tiles + ct - 1) / ct;
+    const long long items = bh * nce;
+    const long long ctas = std::min<long long>(items, num_sms);
+    const long long per = (items + ctas - 1) / ctas;
+    const long long cost = 4 * per * ct + per;
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best_ct = ct;
+    }
+  }
+  return (int)(best_ct * kTileKeys);
 }
 
 size_t decode_smem_bytes(int d, int G, int chunk) {
+  (void)G;
   (void)chunk;
-  if (d == 128) {
-    switch (G) {
-      case 1: return DecSmem<128, 1>::kBytes;
-      case 2: return DecSmem<128, 2>::kBytes;
-      case 4: return DecSmem<128, 4>::kBytes;
-      default: return DecSmem<128, 8>::kBytes;
-    }
-  }
-  switch (G) {
-    case 1: return DecSmem<64, 1>::kBytes;
-    case 2: return DecSmem<64, 2>::kBytes;
-    case 4: return DecSmem<64, 4>::kBytes;
-    default: return DecSmem<64, 8>::kBytes;
-  }
+  return d == 128 ? DecSmem<128>::kBytes : DecSmem<64>::kBytes;
 }
 
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t st) {
@@ -443,15 +595,19 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t st) {
   p.n_keys = a.n_keys;
   p.chunk = a.chunk;
   p.nchunks = decode_num_chunks(a.n_keys, a.chunk);
+  p.item_base = 0;
+  p.num_items = 0;
   p.scale_log2 = a.scale_log2;
   for (int j = 0; j < kMaxHalfDim; ++j) p.inv_freq[j] = j < a.d / 2 ? a.rope.inv_freq[j] : 0.0;
+  if (a.chunk <= 0 || a.chunk % kTileKeys != 0 || a.cache.P % kTileKeys != 0) return cudaErrorInvalidValue;
   CUtensorMap mk, mv;
   if (!make_tile_map(&mk, a.cache.k_pool, a.d, a.cache.P, a.Hkv, a.cache.num_pages) ||
       !make_tile_map(&mv, a.cache.v_pool, a.d, a.cache.P, a.Hkv, a.cache.num_pages))
     return cudaErrorInvalidValue;
   const int G = a.Hq / a.Hkv;
+  const int total = p.nchunks * a.Hkv * a.B;
 #define STAR_DEC_CASE(DD, GG) \
-  if (a.d == DD && G == GG) return launch_dg<DD, GG>(p, mk, mv, st);
+  if (a.d == DD && G == GG) return launch_dg<DD, GG>(p, mk, mv, total, st);
   STAR_DEC_CASE(128, 1)
   STAR_DEC_CASE(128, 2)
   STAR_DEC_CASE(128, 4)

@@ -9,70 +9,101 @@
 // a row with no finite partial gives O = 0, LSE = -inf.
 //
 // One warp per output row; each lane owns d/32 consecutive columns (one
-// 16-byte load per partial at d = 128).  HBM-bound.
+// 16-byte load per partial at d = 128).  The kernel is latency-bound at decode
+// sizes (a few dozen rows), so it keeps memory round trips few: the first batch
+// of O loads is issued before the LSE statistics are read, the statistics are one
+// online (max, sum) pass, and the O partials stream in batches of kBatch loads.
 #include "common.cuh"
 #include "internal.h"
 
 namespace star {
 namespace {
 
+constexpr int kBatch = 16;
+
+template <int D>
+struct Cols;
+template <>
+struct Cols<128> {
+  using T = float4;
+  static __device__ __forceinline__ void fma(float* acc, float w, const T& v) {
+    acc[0] = fmaf(w, v.x, acc[0]);
+    acc[1] = fmaf(w, v.y, acc[1]);
+    acc[2] = fmaf(w, v.z, acc[2]);
+    acc[3] = fmaf(w, v.w, acc[3]);
+  }
+};
+template <>
+struct Cols<64> {
+  using T = float2;
+  static __device__ __forceinline__ void fma(float* acc, float w, const T& v) {
+    acc[0] = fmaf(w, v.x, acc[0]);
+    acc[1] = fmaf(w, v.y, acc[1]);
+  }
+};
+
 template <int D, bool OUT_BF16>
 __global__ void __launch_bounds__(256) lse_merge_kernel(int parts_per_group, long long rows, const float* __restrict__ o_in,
                                                         const float* __restrict__ lse_in, void* __restrict__ o_out,
                                                         float* __restrict__ lse_out) {
   constexpr int PER = D / 32;
+  using V = typename Cols<D>::T;
   const int lane = threadIdx.x % 32;
   const long long row = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   const int group = blockIdx.y;
   if (row >= rows) return;
   const long long part0 = (long long)group * parts_per_group;
   const int np = parts_per_group;
+  const float* ob = o_in + (part0 * rows + row) * D + lane * PER;  // partial i at ob + i * rows * D
+  const float* lb = lse_in + part0 * rows + row;                   // partial i at lb + i * rows
+  const size_t ostride = (size_t)rows * D;
 
-  // LSE statistics: the lanes take the partials 32 at a time.
-  float m = -INFINITY;
+  V v[kBatch];
+#pragma unroll
+  for (int j = 0; j < kBatch; ++j)
+    if (j < np) v[j] = __ldg(reinterpret_cast<const V*>(ob + j * ostride));
+
+  // LSE statistics: online (max, sum) over the lane's partials, then across lanes.
+  float m = -INFINITY, s = 0.f;
   for (int i = lane; i < np; i += 32) {
-    const float li = __ldg(lse_in + (part0 + i) * rows + row);
-    if (isfinite(li)) m = fmaxf(m, li);
+    const float li = __ldg(lb + (size_t)i * rows);
+    if (!isfinite(li)) continue;
+    if (li > m) {
+      s = s * expf(m - li) + 1.f;
+      m = li;
+    } else {
+      s += expf(li - m);
+    }
   }
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  for (int off = 16; off > 0; off >>= 1) {
+    const float mo = __shfl_xor_sync(0xffffffffu, m, off), so = __shfl_xor_sync(0xffffffffu, s, off);
+    const float mm = fmaxf(m, mo);
+    if (mm != -INFINITY) s = (m == -INFINITY ? 0.f : s * expf(m - mm)) + (mo == -INFINITY ? 0.f : so * expf(mo - mm));
+    m = mm;
+  }
+  const float lse = (m == -INFINITY) ? -INFINITY : m + logf(s);
+
   float acc[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
-  float lse = -INFINITY;
   if (m != -INFINITY) {
-    float s = 0.f;
-    for (int i = lane; i < np; i += 32) {
-      const float li = __ldg(lse_in + (part0 + i) * rows + row);
-      if (isfinite(li)) s += expf(li - m);
-    }
+    for (int base = 0; base < np; base += kBatch) {
+      if (base > 0) {
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-    lse = m + logf(s);
-    // O: each lane owns PER consecutive columns; weights are broadcast from the lane
-    // that computed them, and the loads of several partials are in flight at once.
-    for (int base = 0; base < np; base += 32) {
+        for (int j = 0; j < kBatch; ++j)
+          if (base + j < np) v[j] = __ldg(reinterpret_cast<const V*>(ob + (size_t)(base + j) * ostride));
+      }
+      // Lane j holds the weight of partial base + j; a non-finite LSE weighs 0.
       float w = 0.f;
-      if (base + lane < np) {
-        const float li = __ldg(lse_in + (part0 + base + lane) * rows + row);
+      if (lane < kBatch && base + lane < np) {
+        const float li = __ldg(lb + (size_t)(base + lane) * rows);
         if (isfinite(li)) w = expf(li - lse);
       }
-      const int cnt = min(32, np - base);
-#pragma unroll 4
-      for (int j = 0; j < cnt; ++j) {
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
         const float wj = __shfl_sync(0xffffffffu, w, j);
-        const float* src = o_in + ((part0 + base + j) * rows + row) * D + lane * PER;
-        if constexpr (PER == 4) {
-          const float4 v = __ldg(reinterpret_cast<const float4*>(src));
-          acc[0] = fmaf(wj, v.x, acc[0]);
-          acc[1] = fmaf(wj, v.y, acc[1]);
-          acc[2] = fmaf(wj, v.z, acc[2]);
-          acc[3] = fmaf(wj, v.w, acc[3]);
-        } else {
-          const float2 v = __ldg(reinterpret_cast<const float2*>(src));
-          acc[0] = fmaf(wj, v.x, acc[0]);
-          acc[1] = fmaf(wj, v.y, acc[1]);
-        }
+        if (base + j < np) Cols<D>::fma(acc, wj, v[j]);
       }
     }
   }

@@ -59,9 +59,10 @@ def test_noalloc_rejects_shapes_beyond_its_scratch():
         pytest.skip("no CUDA device")
     import block_sparse_attention_star_b200 as star
     from tests import harness
-    # 64 sequences x 64 query heads over a million-token cache: far more decode partials
-    # than the built-in scratch holds (the call is rejected on the host, nothing runs).
-    big = Workload("noalloc-big", B=64, Hq=64, Hkv=8, d=128, L=1 << 20, b=1 << 17, T=32, S=16, peaky=False)
+    # 512 sequences x 64 query heads over a million-token cache: even one chunk per
+    # (sequence, KV head) gives 32768 f32 output rows of 128 values, 16 MiB plus the
+    # LSEs, more than the built-in scratch holds (rejected on the host, nothing runs).
+    big = Workload("noalloc-big", B=512, Hq=64, Hkv=8, d=128, L=1 << 20, b=1 << 17, T=32, S=16, peaky=False)
     shape = harness.shape_of(big)
     assert star.star_workspace_size(shape, star.STAR_OP_DECODE) > 16 << 20
     small = Workload("noalloc-small", B=1, Hq=4, Hkv=1, d=64, L=1024, b=256, T=16, S=2, peaky=False)
