@@ -267,7 +267,7 @@ int star_phase1_encode(const star_shape* shape, const star_cache* cache, const v
   a.L = shape->L;
   a.b = shape->b;
   a.n = shape->n;
-  a.q = q;
+  a.q = out;  // RoPE(q) is staged in the output buffer: each work item reads its Q tile, then writes O there
   a.q_pos = pos_ctx;
   a.Ntok = shape->L;
   a.cache = cv;
@@ -277,7 +277,8 @@ int star_phase1_encode(const star_shape* shape, const star_cache* cache, const v
   a.rope = rt;
   const char* why = nullptr;
   trace_begin(st);
-  e = star::launch_attention(a, st, &why);
+  e = star::launch_rope_q(q, pos_ctx, shape->B, shape->L, shape->Hq, shape->d, out, rt, st);
+  if (e == cudaSuccess) e = star::launch_attention(a, st, &why);
   trace_end(st);
   if (e != cudaSuccess) return why ? fail(STAR_ERR_CUDA, "%s", why) : cuda_fail(e, "phase1 attention launch");
   return STAR_OK;

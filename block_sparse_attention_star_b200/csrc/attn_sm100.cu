@@ -215,7 +215,7 @@ struct Smem {
   static constexpr int kK = 2 * kTile;
   static constexpr int kV = kK + NSK * kTile;
   static constexpr int kBar = kV + NSV * kTile;
-  static constexpr int kNumBars = 2 * NSK + 2 * NSV + 4 * 2 + 1;
+  static constexpr int kNumBars = 2 * NSK + 2 * NSV + 2 + 2 + 4 + 2 + 1 + 2 + 1;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kEnd = kTmemSlot + 16;
   static constexpr int kBytes = kEnd + 1024;  // slack for 1024-byte alignment
@@ -224,7 +224,7 @@ struct Smem {
 template <int D, int MODE, int NSK, int NSV>
 __global__ void __launch_bounds__(kThreads, 1)
     star_attn_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                     const __grid_constant__ Params p) {
+                     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ Params p) {
   using S = Smem<D, MODE, NSK, NSV>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -235,9 +235,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* v_empty = v_full + NSV;
   uint64_t* q_full = v_empty + NSV;   // [2]
   uint64_t* s_full = q_full + 2;      // [2]
-  uint64_t* p_full = s_full + 2;      // [2]
-  uint64_t* o_full = p_full + 2;      // [2]
-  uint64_t* drain = o_full + 2;       // [1]
+  uint64_t* p_full = s_full + 2;      // [2 tiles][2 key halves]
+  uint64_t* o_full = p_full + 4;      // [2]
+  uint64_t* q_empty = o_full + 2;     // [1] mode 0: the item's last Q K^T is done
+  uint64_t* o_free = q_empty + 1;     // [2] mode 0: the epilogue has read O_w
+  uint64_t* drain = o_free + 2;       // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kTmemSlot);
 
   const int warp = threadIdx.x / 32;
@@ -247,17 +249,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < NSK; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1); }
     for (int s = 0; s < NSV; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1); }
     for (int w = 0; w < 2; ++w) {
-      mbar_init(&q_full[w], kRows);
+      mbar_init(&q_full[w], MODE == 0 ? 1 : kRows);  // mode 0: TMA bytes; mode 1: every row's thread
+      mbar_init(&o_free[w], 4);
       mbar_init(&s_full[w], 1);
-      mbar_init(&p_full[w], kRows);
+      mbar_init(&p_full[2 * w], 4);
+      mbar_init(&p_full[2 * w + 1], 4);
       mbar_init(&o_full[w], 1);
     }
+    mbar_init(q_empty, 1);
     mbar_init(drain, 1);
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
+    if (MODE == 0) prefetch_tmap(&tmQ);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -319,6 +325,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(&v_full[s], (last / NSV) & 1, kDevTimeoutProducer);
       }
     }
+  } else if (MODE == 0 && warp == 3) {
+    // ------------------------------------------------------------------ Q producer (mode 0)
+    // The two Q tiles of each item (rows r0 .. r0 + 127 of two query heads, already
+    // rotated) by TMA, as soon as the previous item's last Q K^T has completed.
+    if (lane == 0) {
+      uint32_t qc = 0;
+      bool ok = true;
+      for (int idx = blockIdx.x; idx < p.num_items && ok; idx += gridDim.x, ++qc) {
+        const Item it = decode_item<MODE>(p, idx);
+        if (qc > 0) ok = mbar_wait(q_empty, (qc - 1) & 1, kDevTimeoutProducer);
+        if (!ok) break;
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          mbar_arrive_expect_tx(&q_full[w], S::kTile);
+#pragma unroll
+          for (int h = 0; h < D / 64; ++h)
+            tma_load_4d(smem + S::kQ0 + w * S::kTile + h * (kRows * 128), &tmQ, &q_full[w], h * 64,
+                        it.g * p.G + 2 * it.hp + w, it.r0, it.bi);
+        }
+      }
+      // Drain: the last loads have landed before the CTA exits.
+      if (qc > 0) {
+        mbar_wait(&q_full[0], (qc - 1) & 1, kDevTimeoutProducer);
+        mbar_wait(&q_full[1], (qc - 1) & 1, kDevTimeoutProducer);
+      }
+    }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -327,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sQ = smem_u32(smem + S::kQ0);
       const uint32_t sK = smem_u32(smem + S::kK);
       const uint32_t sV = smem_u32(smem + S::kV);
-      uint32_t kcnt = 0, vcnt = 0, qph = 0, pph[2] = {0, 0};
+      uint32_t kcnt = 0, vcnt = 0, qph = 0, pph[4] = {0, 0, 0, 0};
       bool ok = true;
       bool issued = false;
 
@@ -345,13 +377,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       // O_w += P_w V: P from TMEM (8 columns per 16 keys); V MN-major (d contiguous),
       // 8 keys of 128 B per swizzle group (SBO 1024 B), 64-column d atoms 16 KB apart (LBO).
-      auto issue_pv = [&](int w, int vs, bool acc) {
+      // Issued per 64-key half as soon as the softmax has stored that half of P_w,
+      // so the first half's product overlaps the second half's exponentials.
+      uint32_t nitem = 0;
+      auto issue_pv = [&](int w, int vs, bool acc) -> bool {
         const uint32_t vb = sV + vs * S::kTile;
+        // Mode 0: the first product of an item overwrites O_w, which the previous
+        // item's epilogue must have read.
+        if (MODE == 0 && !acc && nitem > 0 && !mbar_wait(&o_free[w], (nitem - 1) & 1, kDevTimeoutMma)) return false;
 #pragma unroll
-        for (int kk = 0; kk < kKeys / 16; ++kk) {
-          mma_ts(tbase + 256 + w * 128, tbase + w * 128 + kk * 8, umma_desc_sw128(vb + kk * 2048, kKeys * 128, 1024),
-                 idesc_pv, (acc || kk > 0) ? 1u : 0u);
+        for (int half = 0; half < 2; ++half) {
+          if (!mbar_wait(&p_full[2 * w + half], pph[2 * w + half], kDevTimeoutMma)) return false;
+          pph[2 * w + half] ^= 1;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = half * 4; kk < half * 4 + 4; ++kk)
+            mma_ts(tbase + 256 + w * 128, tbase + w * 128 + kk * 8,
+                   umma_desc_sw128(vb + kk * 2048, kKeys * 128, 1024), idesc_pv, (acc || kk > 0) ? 1u : 0u);
         }
+        return true;
       };
 
       for (int idx = blockIdx.x; idx < p.num_items && ok; idx += gridDim.x) {
@@ -368,51 +412,37 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           int vs = 0;
           if (j > 0) {
-            ok = mbar_wait(&p_full[0], pph[0], kDevTimeoutMma);
-            if (!ok) break;
-            pph[0] ^= 1;
             vs = vcnt % NSV;
-            ok = mbar_wait(&v_full[vs], (vcnt / NSV) & 1, kDevTimeoutMma);
+            ok = mbar_wait(&v_full[vs], (vcnt / NSV) & 1, kDevTimeoutMma) && issue_pv(0, vs, j > 1);
             if (!ok) break;
-            tc_fence_after();
-            issue_pv(0, vs, j > 1);
           }
           issue_s(0, ks);
           issued = true;
           mma_commit(&s_full[0]);
           if (j > 0) {
-            ok = mbar_wait(&p_full[1], pph[1], kDevTimeoutMma);
+            ok = issue_pv(1, vs, j > 1);
             if (!ok) break;
-            pph[1] ^= 1;
-            tc_fence_after();
-            issue_pv(1, vs, j > 1);
             mma_commit(&v_empty[vs]);
             ++vcnt;
           }
           issue_s(1, ks);
           mma_commit(&s_full[1]);
           mma_commit(&k_empty[ks]);
+          if (MODE == 0 && j == nt - 1) mma_commit(q_empty);
           ++kcnt;
         }
         if (!ok) break;
         // The last tile's P V products.
-        ok = mbar_wait(&p_full[0], pph[0], kDevTimeoutMma);
-        if (!ok) break;
-        pph[0] ^= 1;
         const int vs = vcnt % NSV;
-        ok = mbar_wait(&v_full[vs], (vcnt / NSV) & 1, kDevTimeoutMma);
+        ok = mbar_wait(&v_full[vs], (vcnt / NSV) & 1, kDevTimeoutMma) && issue_pv(0, vs, nt > 1);
         if (!ok) break;
-        tc_fence_after();
-        issue_pv(0, vs, nt > 1);
         mma_commit(&o_full[0]);
-        ok = mbar_wait(&p_full[1], pph[1], kDevTimeoutMma);
+        ok = issue_pv(1, vs, nt > 1);
         if (!ok) break;
-        pph[1] ^= 1;
-        tc_fence_after();
-        issue_pv(1, vs, nt > 1);
         mma_commit(&v_empty[vs]);
         ++vcnt;
         mma_commit(&o_full[1]);
+        ++nitem;
       }
       if (issued) {
         // Every MMA this thread issued has completed before TMEM is released.
@@ -439,16 +469,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       {
         const Item it = decode_item<MODE>(p, idx);
         const RowInfo ri = row_info<MODE>(p, it, wg, row);
-        load_q_row<D>(p, it, ri, sQ, row);
+        if (MODE == 1) load_q_row<D>(p, it, ri, sQ, row);  // mode 0: Q arrives by TMA
         nt = it.a_tiles + it.b_tiles;
         a_tiles = it.a_tiles;
         a_start = it.a_start;
         b_start = it.b_start;
         cache_idx = ri.cache_idx;
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(&q_full[wg]);
+      if (MODE == 1) {
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&q_full[wg]);
+      }
 
       float m = -INFINITY, l = 0.f, lr = 0.f;
       for (int j = 0; j < nt; ++j) {
@@ -470,9 +502,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Row max of the raw scores (scale > 0 commutes with max); 4 independent chains.
         float mx[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) mx[e] = __uint_as_float(sr[e]);
+        for (int e = 0; e < 4; ++e) mx[e] = fmaxf(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]));
 #pragma unroll
-        for (int c = 4; c < kKeys; ++c) mx[c % 4] = fmaxf(mx[c % 4], __uint_as_float(sr[c]));
+        for (int c = 8; c < kKeys; c += 8)
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            mx[e] = fmax3(mx[e], __uint_as_float(sr[c + 2 * e]), __uint_as_float(sr[c + 2 * e + 1]));
         const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
         const float m_new = fmaxf(m, mt * p.scale_log2);
         float f = 1.f;
@@ -482,12 +517,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           m = m_new;
         }
         const float mu = (m == -INFINITY) ? 0.f : m;
+        // tcgen05.ld/st are warp-collective (.sync.aligned): the whole warp takes
+        // this branch when any of its rows must rescale; the others scale by 1.
+        // O_w holds the products of tiles < j only (s_full of tile j is committed
+        // after the P V of tile j - 1), so it can be scaled in place; 8 columns at a
+        // time, since the 128 scores of the row are live here.
+        if (__any_sync(0xffffffffu, f != 1.f)) {
+#pragma unroll 1
+          for (int c = 0; c < D / 8; ++c) {
+            uint32_t o[8];
+            tmem_ld8(tO + c * 8, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 8; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+            tmem_st8(tO + c * 8, o);
+          }
+        }
         // P = 2^(s*scale - m) (exponent arguments two at a time), rounded to bf16 for
         // the P V product; l sums the f32 values (the log-sum-exp needs no bf16
-        // rounding in it).  P is written to TMEM in two 32-column halves.
+        // rounding in it), two at a time.  Each 64-key half of P goes to TMEM (32
+        // columns) and is handed to the MMA warp before the next half is computed.
         const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
         const uint64_t nm2 = f2_pack(-mu, -mu);
-        float su[2] = {0.f, 0.f};
+        uint64_t su2[2] = {0ull, 0ull};
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t pk[32];
@@ -498,11 +550,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * cc]), __uint_as_float(sr[2 * cc + 1])), sc2, nm2), x0, x1);
             const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
             pk[c] = pack_bf16x2(p0, p1);
-            su[c & 1] += p0 + p1;
+            su2[c & 1] = f2_add(su2[c & 1], f2_pack(p0, p1));
           }
           tmem_st32(tS + half * 32, pk);
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&p_full[2 * wg + half]);
         }
-        const float rs_u = su[0] + su[1];
+        float s0, s1, s2, s3;
+        f2_unpack(su2[0], s0, s1);
+        f2_unpack(su2[1], s2, s3);
+        const float rs_u = (s0 + s1) + (s2 + s3);
         // O is normalised by the sum of the bf16-rounded P so that it stays a convex
         // combination of V rows when one key dominates; the rounding that matters
         // there is the largest P's, so its error is added to the f32 sum.
@@ -510,24 +569,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float rs_r = rs_u + (__bfloat162float(__float2bfloat16_rn(pmax)) - pmax);
         l = l * f + rs_u;
         lr = lr * f + rs_r;
-        // tcgen05.ld/st are warp-collective (.sync.aligned): the whole warp takes
-        // this branch when any of its rows must rescale; the others scale by 1.
-        if (__any_sync(0xffffffffu, f != 1.f)) {
-          // O_w holds the products of tiles < j only (its P V for tile j is not
-          // issued before p_full), so it can be scaled in place.
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tO + c * 32, o);
-            tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-            tmem_st32(tO + c * 32, o);
-          }
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&p_full[wg]);
       }
       if (!ok) break;
       ok = __all_sync(0xffffffffu, mbar_wait(&o_full[wg], oph, kDevTimeoutSoftmax));
@@ -552,6 +593,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) d4[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
         }
+        // O_w is read: the next item's first P V may overwrite it.
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&o_free[wg]);
       } else {
         const size_t rowoff = (((size_t)it.part * p.B + it.bi) * p.Ntok + ri.tok) * p.Hq + ri.head;
         float* dst = p.out_f32 + rowoff * D;
@@ -619,6 +664,20 @@ bool make_pool_map(CUtensorMap* map, void* pool, int d, int P, int Hkv, int num_
   return r == CUDA_SUCCESS;
 }
 
+// Rotated queries [B][L][Hq][d] bf16 as a 4-D tensor (d innermost); box = 64 x 1 head x 128 rows x 1.
+bool make_q_map(CUtensorMap* map, const void* q, int d, int Hq, int L, int B) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)Hq, (cuuint64_t)L, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)Hq * d * 2, (cuuint64_t)L * Hq * d * 2};
+  const cuuint32_t box[4] = {64, 1, (cuuint32_t)kRows, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(q), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int pow2_at_least(int x) {
   int v = 1;
   while (v < x) v <<= 1;
@@ -627,7 +686,7 @@ int pow2_at_least(int x) {
 
 template <int D, int MODE>
 cudaError_t launch_typed(const AttnLaunch& a, const Params& p, const CUtensorMap& mk, const CUtensorMap& mv,
-                         cudaStream_t st) {
+                         const CUtensorMap& mq, cudaStream_t st) {
   constexpr int NSK = (D == 128) ? 2 : 4;
   constexpr int NSV = (D == 128) ? 2 : 4;
   using S = Smem<D, MODE, NSK, NSV>;
@@ -643,7 +702,7 @@ cudaError_t launch_typed(const AttnLaunch& a, const Params& p, const CUtensorMap
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = std::min(p.num_items, sms);
   if (grid <= 0) return cudaSuccess;
-  kern<<<grid, kThreads, S::kBytes, st>>>(mk, mv, p);
+  kern<<<grid, kThreads, S::kBytes, st>>>(mk, mv, mq, p);
   return cudaGetLastError();
 }
 
@@ -692,10 +751,15 @@ cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t st, const char** 
     if (why) *why = "cuTensorMapEncodeTiled failed for the KV pools";
     return cudaErrorInvalidValue;
   }
+  CUtensorMap mq = mk;  // mode 1 stages Q with its own threads; the map is unused there
+  if (a.mode == 0 && !make_q_map(&mq, a.q, a.d, a.Hq, a.L, a.B)) {
+    if (why) *why = "cuTensorMapEncodeTiled failed for the rotated queries";
+    return cudaErrorInvalidValue;
+  }
   if (a.d == 128) {
-    return a.mode == 0 ? launch_typed<128, 0>(a, p, mk, mv, st) : launch_typed<128, 1>(a, p, mk, mv, st);
+    return a.mode == 0 ? launch_typed<128, 0>(a, p, mk, mv, mq, st) : launch_typed<128, 1>(a, p, mk, mv, mq, st);
   } else {
-    return a.mode == 0 ? launch_typed<64, 0>(a, p, mk, mv, st) : launch_typed<64, 1>(a, p, mk, mv, st);
+    return a.mode == 0 ? launch_typed<64, 0>(a, p, mk, mv, mq, st) : launch_typed<64, 1>(a, p, mk, mv, mq, st);
   }
 }
 

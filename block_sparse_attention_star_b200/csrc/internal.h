@@ -28,6 +28,10 @@ struct CacheView {
 // slots [start, start + ntok).  k/v: [B][ntok][Hkv][d] bf16, pos: [B][ntok].
 cudaError_t launch_rope_append(const void* k, const void* v, const int32_t* pos, int B, int ntok, int start,
                                int Hkv, int d, const CacheView& c, const RopeTable& rt, cudaStream_t st);
+// RoPE of all H query heads of ntok tokens: out = rotate(q) at pos (out may be q).
+// q/out: [B][ntok][H][d] bf16, pos: [B][ntok].
+cudaError_t launch_rope_q(const void* q, const int32_t* pos, int B, int ntok, int H, int d, void* out,
+                          const RopeTable& rt, cudaStream_t st);
 // Zero cache slots [from, to) of every sequence (K and V).
 cudaError_t launch_zero_slots(int B, int from, int to, int Hkv, int d, const CacheView& c, cudaStream_t st);
 // c' position ids [B][L + (n-1) b] and block map [B][L][3].
@@ -44,7 +48,7 @@ cudaError_t launch_lse_merge(int groups, int parts_per_group, int64_t rows, int 
 struct AttnLaunch {
   int mode;               // 0: Phase-1 context attention, 1: Phase-2 query partials
   int B, Hq, Hkv, d, L, b, n;
-  const void* q;          // [B][Ntok][Hq][d] bf16 (pre-RoPE)
+  const void* q;          // [B][Ntok][Hq][d] bf16: mode 0 already rotated (staged by TMA), mode 1 pre-RoPE
   const int32_t* q_pos;   // [B][Ntok]
   int Ntok;
   CacheView cache;

@@ -10,6 +10,8 @@
 // * zero_slots: clears cache slots past the context so that tiles which run over
 //   the valid tail hold zeros, not stale values (masked keys get P = 0, and
 //   0 * V must stay 0).
+// * rope_q: the query heads rotated by RoPE once, before the attention kernel
+//   (which then stages Q tiles by TMA instead of rotating them per work item).
 // * build_positions: the integer position ids of c' and the token -> (block,
 //   page, slot) map ("被增广的上下文").
 //
@@ -71,6 +73,42 @@ __global__ void __launch_bounds__(256) rope_append_kernel(const bf16* __restrict
       *reinterpret_cast<uint4*>(vpool + dst + 8 * c) = __ldg(reinterpret_cast<const uint4*>(v + src + 8 * c));
       *reinterpret_cast<uint4*>(vpool + dst + D / 2 + 8 * c) =
           __ldg(reinterpret_cast<const uint4*>(v + src + D / 2 + 8 * c));
+    }
+  }
+}
+
+// RoPE of the query heads of ntok tokens per sequence: out[b][t][h] = rotation of
+// q[b][t][h] at pos[b][t] (float64 rotation, one bf16 rounding, as the keys).  One
+// thread per (sequence, token, 8-pair chunk): the 8 angles are computed once and
+// applied to that chunk of every query head.  out may be q itself: each element is
+// read and then written by the same thread.
+template <int D>
+__global__ void __launch_bounds__(256) rope_q_kernel(const bf16* q, const int32_t* __restrict__ pos, int B, int ntok,
+                                                     int H, bf16* out, const __grid_constant__ RopeParams rp) {
+  constexpr int CH = D / 16;
+  const long long total = (long long)B * ntok * CH;
+  for (long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x; gid < total;
+       gid += (long long)gridDim.x * blockDim.x) {
+    const int c = (int)(gid % CH);
+    const long long r = gid / CH;  // bi * ntok + t
+    const int p_t = pos[r];
+    double cs[4][2], sn[4][2];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      rope_sincos(p_t, rp.inv_freq[8 * c + 2 * e], cs[e][0], sn[e][0]);
+      rope_sincos(p_t, rp.inv_freq[8 * c + 2 * e + 1], cs[e][1], sn[e][1]);
+    }
+    for (int h = 0; h < H; ++h) {
+      const size_t off = ((size_t)r * H + h) * D;
+      const uint4 a = *reinterpret_cast<const uint4*>(q + off + 8 * c);
+      const uint4 bq = *reinterpret_cast<const uint4*>(q + off + D / 2 + 8 * c);
+      const uint32_t* aw = reinterpret_cast<const uint32_t*>(&a);
+      const uint32_t* bw = reinterpret_cast<const uint32_t*>(&bq);
+      uint32_t lo[4], hi[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) rope_rotate2(aw[e], bw[e], cs[e], sn[e], lo[e], hi[e]);
+      *reinterpret_cast<uint4*>(out + off + 8 * c) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      *reinterpret_cast<uint4*>(out + off + D / 2 + 8 * c) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
     }
   }
 }
@@ -160,6 +198,22 @@ cudaError_t launch_rope_append(const void* k, const void* v, const int32_t* pos,
         reinterpret_cast<bf16*>(c.k_pool), reinterpret_cast<bf16*>(c.v_pool), c.page_table, c.max_pages,
         c.num_pages, c.P, rp);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope_q(const void* q, const int32_t* pos, int B, int ntok, int H, int d, void* out,
+                          const RopeTable& rt, cudaStream_t st) {
+  if (ntok <= 0 || B <= 0) return cudaSuccess;
+  RopeParams rp;
+  for (int j = 0; j < d / 2; ++j) rp.inv_freq[j] = rt.inv_freq[j];
+  const long long work = (long long)B * ntok * (d / 16);
+  const int grid = grid_for(work, 256);
+  if (d == 128)
+    rope_q_kernel<128><<<grid, 256, 0, st>>>(reinterpret_cast<const bf16*>(q), pos, B, ntok, H,
+                                             reinterpret_cast<bf16*>(out), rp);
+  else
+    rope_q_kernel<64><<<grid, 256, 0, st>>>(reinterpret_cast<const bf16*>(q), pos, B, ntok, H,
+                                            reinterpret_cast<bf16*>(out), rp);
   return cudaGetLastError();
 }
 

@@ -129,7 +129,9 @@ int star_kv_append(const star_shape* shape, const star_cache* cache, const void*
  * keys [0, b) (for i > 1) and to its own block's keys up to t, each key roped at
  * its own position id.  Writes RoPE(K), V of the L context tokens into cache
  * slots [0, L) (the anchor copies are never written) and zeroes slots
- * [L, L + round_up(T_max,128)).
+ * [L, L + round_up(T_max,128)).  out also serves as the staging buffer of RoPE(q)
+ * during the call (each row is rotated there, then overwritten by its output), so
+ * out may be q itself but must not partly overlap q, k or v.
  * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, ALIGNMENT, CAPACITY, CUDA. */
 int star_phase1_encode(const star_shape* shape, const star_cache* cache, const void* q, const void* k,
                        const void* v, const int32_t* pos_ctx, void* out, void* ws, size_t ws_bytes,
