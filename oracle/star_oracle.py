@@ -42,10 +42,15 @@ Parity status per function (the pins live in ``tests/test_oracle_pins.py``):
 * ``round_to_bf16``          pinned: hand-computed ties; torch's fp32->bf16 cast on fp32-exact inputs.
 * ``rope_inv_freq``/``apply_rope`` pinned: complex-multiplication form, norm and
   relative-shift invariance, identity at position 0, closed-form angles.
-* ``augmented_context``/``block_map`` pinned: hand-enumerated L=8, b=2 fixture.
+* ``augmented_context``/``block_map`` pinned: hand-enumerated L=8, b=2 fixture; the
+  anchor variants (anchor size a < b, per-block anchor position ids) by the
+  hand-enumerated L=12, b=4, a=2 fixture.
 * ``causal_attention``       pinned: torch scaled_dot_product_attention (causal, fp64).
 * ``phase1``/``phase1_rows`` pinned: n=1 equals textbook causal attention; n>1
-  equals an independent full-length attention with the Star mask (library SDPA).
+  equals an independent full-length attention with the Star mask (library SDPA);
+  with anchor variants, equals attention over each row's explicitly built key set
+  (anchor keys roped at the anchor ids, own-block keys up to the row), and a
+  common shift of all position ids leaves the outputs unchanged up to rounding.
 * ``attend``/``phase2_partials``/``lse_merge``/``decode_step`` pinned: the merge
   equals brute-force softmax over the concatenated cache (library SDPA and
   scipy logsumexp); merge identities and overflow cases in closed form.
@@ -125,7 +130,7 @@ def rope_bf16(x: np.ndarray, pos, theta: float) -> np.ndarray:
 # Phase 1 structure: the augmented context c' and the block map
 # ----------------------------------------------------------------------------
 
-def augmented_context(L: int, b: int, pos_ctx=None) -> list[dict]:
+def augmented_context(L: int, b: int, pos_ctx=None, anchor: int | None = None, anchor_pos=None) -> list[dict]:
     """c' = [c_1, (c_1 c_2), ..., (c_1 c_n)] with its position ids.
 
     [SA1] "Phase 1: 被增广的上下文": every block after the first is prefixed by
@@ -133,19 +138,36 @@ def augmented_context(L: int, b: int, pos_ctx=None) -> list[dict]:
     0..b-1), while c_i keeps its own ids [(i-1)b, ib).  [SA1] "局部注意力与 KV
     丢弃": only the c_i part's KV is kept.
 
+    Anchor variants ([SA1] "仓库里的真实实现": the anchor size is a parameter of
+    its own, by default the whole first block; the implementers' notes on the
+    anchor's position ids: ids sampled from the prefix range, or reset to 0):
+    ``anchor`` = a <= b takes the first a tokens of c_1 as the anchor;
+    ``anchor_pos`` [n-1, a] gives the anchor's position ids in block i >= 1
+    (0-based), default the caller's ids of tokens 0..a-1.
+
     Returns one dict per block (0-based ``i``) with ``tokens`` (context token
     index of every augmented row), ``pos`` (its position id) and ``kept`` (the
     augmented rows whose output and KV survive).
     """
     if L % b:
         raise ValueError("context length must be a multiple of the block size")
+    a = b if anchor is None else int(anchor)
+    if not 0 < a <= b:
+        raise ValueError("anchor size must be in (0, b]")
+    n = L // b
     pos_ctx = np.arange(L, dtype=np.int64) if pos_ctx is None else np.asarray(pos_ctx, dtype=np.int64)
+    if anchor_pos is not None:
+        anchor_pos = np.asarray(anchor_pos, dtype=np.int64).reshape(n - 1, a)
     out = []
-    for i in range(L // b):
+    for i in range(n):
         own = np.arange(i * b, (i + 1) * b, dtype=np.int64)
-        tokens = own if i == 0 else np.concatenate([np.arange(b, dtype=np.int64), own])
-        out.append({"i": i, "tokens": tokens, "pos": pos_ctx[tokens],
-                    "kept": np.arange(len(tokens) - b, len(tokens))})
+        if i == 0:
+            tokens, pos = own, pos_ctx[own]
+        else:
+            tokens = np.concatenate([np.arange(a, dtype=np.int64), own])
+            apos = pos_ctx[:a] if anchor_pos is None else anchor_pos[i - 1]
+            pos = np.concatenate([apos, pos_ctx[own]])
+        out.append({"i": i, "tokens": tokens, "pos": pos, "kept": np.arange(len(tokens) - b, len(tokens))})
     return out
 
 
@@ -202,18 +224,20 @@ def causal_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray):
 # Phase 1
 # ----------------------------------------------------------------------------
 
-def phase1(q: np.ndarray, k: np.ndarray, v: np.ndarray, pos_ctx, b: int, theta: float):
+def phase1(q: np.ndarray, k: np.ndarray, v: np.ndarray, pos_ctx, b: int, theta: float,
+           anchor: int | None = None, anchor_pos=None):
     """Phase 1 of one sequence by literally building c'.
 
     q [L, Hq, d], k/v [L, Hkv, d] (pre-RoPE, bf16 values held in float64).
     Returns O_ctx [L, Hq, d] (float64), and the cache: roped bf16 K [L, Hkv, d]
     and V [L, Hkv, d] -- only the c_i parts, the anchor copies are dropped.
+    ``anchor``/``anchor_pos``: the anchor variants of ``augmented_context``.
     """
     L = q.shape[0]
     O = np.zeros_like(q, dtype=np.float64)
     ck = np.zeros_like(k, dtype=np.float64)
     cv = np.zeros_like(v, dtype=np.float64)
-    for blk in augmented_context(L, b, pos_ctx):
+    for blk in augmented_context(L, b, pos_ctx, anchor, anchor_pos):
         tok, pos, kept = blk["tokens"], blk["pos"], blk["kept"]
         qr = rope_bf16(q[tok], pos, theta)
         kr = rope_bf16(k[tok], pos, theta)
@@ -226,16 +250,23 @@ def phase1(q: np.ndarray, k: np.ndarray, v: np.ndarray, pos_ctx, b: int, theta: 
     return O, ck, cv
 
 
-def phase1_rows(rows, q_rows: np.ndarray, k: np.ndarray, v: np.ndarray, pos_ctx, b: int, theta: float):
+def phase1_rows(rows, q_rows: np.ndarray, k: np.ndarray, v: np.ndarray, pos_ctx, b: int, theta: float,
+                anchor: int | None = None, anchor_pos=None):
     """Phase-1 outputs of selected context rows only (same definition as ``phase1``).
 
     rows: context token indices; q_rows [len(rows), Hq, d] their pre-RoPE queries;
     k/v [L, Hkv, d] the context keys/values.  Row t of block i = t // b is the
-    augmented row of c'_i that holds token t; it sees the augmented rows before it.
+    augmented row of c'_i that holds token t; it sees the augmented rows before it:
+    the whole anchor (its first a tokens, roped at the anchor's ids) and its own
+    block up to t.
     """
     rows = np.asarray(rows, dtype=np.int64)
     L = k.shape[0]
+    n = L // b
+    a = b if anchor is None else int(anchor)
     pos_ctx = np.arange(L, dtype=np.int64) if pos_ctx is None else np.asarray(pos_ctx, dtype=np.int64)
+    if anchor_pos is not None:
+        anchor_pos = np.asarray(anchor_pos, dtype=np.int64).reshape(n - 1, a)
     out = np.zeros((len(rows),) + q_rows.shape[1:])
     cache: dict[int, np.ndarray] = {}
 
@@ -250,9 +281,10 @@ def phase1_rows(rows, q_rows: np.ndarray, k: np.ndarray, v: np.ndarray, pos_ctx,
         own = np.arange(i * b, (i + 1) * b)
         keys, vals, key_idx = roped_block(i), np.asarray(v[own], dtype=np.float64), own
         if i > 0:
-            keys = np.concatenate([roped_block(0), keys])
-            vals = np.concatenate([np.asarray(v[:b], dtype=np.float64), vals])
-            key_idx = np.concatenate([np.arange(b), own])
+            apos = pos_ctx[:a] if anchor_pos is None else anchor_pos[i - 1]
+            keys = np.concatenate([rope_bf16(k[:a], apos, theta), keys])
+            vals = np.concatenate([np.asarray(v[:a], dtype=np.float64), vals])
+            key_idx = np.concatenate([np.arange(a), own])
         # augmented row of token t sees the anchor (all of it) and its own block up to t
         vis = key_idx[None, :] <= rows[sel][:, None]
         qr = rope_bf16(q_rows[sel], pos_ctx[rows[sel]], theta)
@@ -345,20 +377,24 @@ def decode_step(q_tok: np.ndarray, k_tok: np.ndarray, v_tok: np.ndarray, pos, ck
 # The whole path for one workload
 # ----------------------------------------------------------------------------
 
-def run_star(inp: dict, L: int, b: int, theta: float, with_phase1: bool = True) -> dict:
+def run_star(inp: dict, L: int, b: int, theta: float, with_phase1: bool = True, anchor: int | None = None) -> dict:
     """Phase 1, Phase 2 (partials + merge) and decode for every sequence.
 
     ``inp`` holds float64 (bf16-valued) arrays laid out like the synthetic inputs:
     q_ctx [B, L, Hq, d], k_ctx/v_ctx [B, L, Hkv, d], pos_ctx [B, L], q_query
     [B, T, Hq, d], k_query/v_query [B, T, Hkv, d], pos_query [B, T], q_dec
-    [S, B, 1, Hq, d], k_dec/v_dec [S, B, 1, Hkv, d], pos_dec [S, B].
+    [S, B, 1, Hq, d], k_dec/v_dec [S, B, 1, Hkv, d], pos_dec [S, B]; optionally
+    anchor_pos [B, n-1, a] (the anchor's position ids per block, see
+    ``augmented_context``).  ``anchor``: the anchor size a (default b).
     """
     B = inp["q_ctx"].shape[0]
     res: dict[str, list] = {k: [] for k in ("o_ctx", "cache_k", "cache_v", "o_part", "lse_part",
                                             "o_query", "lse_query", "o_dec", "lse_dec")}
     for bi in range(B):
         if with_phase1:
-            O1, ck, cv = phase1(inp["q_ctx"][bi], inp["k_ctx"][bi], inp["v_ctx"][bi], inp["pos_ctx"][bi], b, theta)
+            apos = inp["anchor_pos"][bi] if inp.get("anchor_pos") is not None else None
+            O1, ck, cv = phase1(inp["q_ctx"][bi], inp["k_ctx"][bi], inp["v_ctx"][bi], inp["pos_ctx"][bi], b, theta,
+                                anchor, apos)
             res["o_ctx"].append(O1)
         else:
             tok = np.arange(L)

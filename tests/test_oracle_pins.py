@@ -375,8 +375,8 @@ def _star_pin_holds():
 def test_planted_wrong_anchor_positions_is_caught(monkeypatch):
     real = oracle.star_oracle.augmented_context
 
-    def shifted(L, b, pos_ctx=None):
-        blocks = real(L, b, pos_ctx)
+    def shifted(L, b, pos_ctx=None, anchor=None, anchor_pos=None):
+        blocks = real(L, b, pos_ctx, anchor, anchor_pos)
         for blk in blocks[1:]:
             blk["pos"] = blk["pos"].copy()
             blk["pos"][:b] += blk["i"] * b - b        # anchor placed just before c_i
@@ -389,8 +389,8 @@ def test_planted_wrong_anchor_positions_is_caught(monkeypatch):
 def test_planted_missing_anchor_is_caught(monkeypatch):
     real = oracle.star_oracle.augmented_context
 
-    def no_anchor(L, b, pos_ctx=None):
-        blocks = real(L, b, pos_ctx)
+    def no_anchor(L, b, pos_ctx=None, anchor=None, anchor_pos=None):
+        blocks = real(L, b, pos_ctx, anchor, anchor_pos)
         for blk in blocks[1:]:
             blk["tokens"], blk["pos"] = blk["tokens"][b:], blk["pos"][b:]
             blk["kept"] = np.arange(b)
@@ -422,3 +422,128 @@ def test_planted_merge_without_rescale_is_caught(monkeypatch):
     monkeypatch.setattr(oracle, "lse_merge", naive)
     with pytest.raises(AssertionError):
         test_lse_merge_of_partials_equals_brute_force()
+
+
+# ---------------------------------------------------------------------------
+# Anchor variants: anchor size a < b and the anchor's position ids
+# ---------------------------------------------------------------------------
+
+def star_mask_anchor(L, b, a):
+    """Full-length visibility with an anchor of the first a tokens."""
+    t = np.arange(L)
+    same_block = (t[:, None] // b) == (t[None, :] // b)
+    causal = t[None, :] <= t[:, None]
+    return (same_block & causal) | ((t[None, :] < a) & (t[:, None] >= b))
+
+
+def test_anchor_variants_match_hand_fixture():
+    g = _golden("anchor_L12_b4_a2.json")
+    for name, var in g["variants"].items():
+        blocks = oracle.augmented_context(g["L"], g["b"], None, g["a"], var["anchor_pos"])
+        assert [blk["tokens"].tolist() for blk in blocks] == g["augmented_tokens"], name
+        assert [blk["pos"].tolist() for blk in blocks] == var["augmented_pos"], name
+        assert [blk["kept"].tolist() for blk in blocks] == g["kept"], name
+        kept = np.concatenate([blk["tokens"][blk["kept"]] for blk in blocks])
+        assert kept.tolist() == g["cached_tokens"]
+        assert sum(len(blk["tokens"]) - len(blk["kept"]) for blk in blocks) == g["anchor_rows_dropped"]
+    assert star_mask_anchor(g["L"], g["b"], g["a"]).astype(int).tolist() == g["star_visibility"]
+
+
+def _anchor_case(seed, L=48, b=16, a=8, Hq=4, Hkv=2, d=16):
+    rng = np.random.default_rng(seed)
+    q, k, v = _bf16_values(rng, (L, Hq, d)), _bf16_values(rng, (L, Hkv, d)), _bf16_values(rng, (L, Hkv, d))
+    n = L // b
+    offs = np.array([rng.integers(0, i * b - a + 1) for i in range(1, n)])
+    variants = {
+        "context": np.tile(np.arange(a), (n - 1, 1)),
+        "offset": offs[:, None] + np.arange(a)[None, :],
+        "zero": np.zeros((n - 1, a), dtype=np.int64),
+    }
+    return q, k, v, variants
+
+
+def explicit_anchor_phase1(q, k, v, pos, b, a, anchor_pos, theta):
+    """Phase 1 built per block from each row's key set: the anchor's first a keys roped at the
+    anchor ids (complex-multiplication RoPE, rounded), then the block's own keys up to the row."""
+    L = q.shape[0]
+    out = np.zeros_like(q)
+    qr = oracle.round_to_bf16(rope_complex(q, pos, theta))
+    kr = oracle.round_to_bf16(rope_complex(k, pos, theta))
+    for i in range(L // b):
+        own = np.arange(i * b, (i + 1) * b)
+        causal = np.tril(np.ones((b, b), dtype=bool))
+        if i == 0:
+            out[own] = sdpa(qr[own], kr[own], v[own], causal)
+            continue
+        ka = oracle.round_to_bf16(rope_complex(k[:a], anchor_pos[i - 1], theta))
+        keys = np.concatenate([ka, kr[own]])
+        vals = np.concatenate([v[:a], v[own]])
+        mask = np.concatenate([np.ones((b, a), dtype=bool), causal], axis=1)
+        out[own] = sdpa(qr[own], keys, vals, mask)
+    return out
+
+
+def test_phase1_anchor_variants_equal_explicit_key_sets():
+    theta = 500000.0
+    q, k, v, variants = _anchor_case(21)
+    L, b, a = q.shape[0], 16, 8
+    pos = np.arange(L)
+    for name, apos in variants.items():
+        O, ck, cv = oracle.phase1(q, k, v, pos, b, theta, a, apos)
+        np.testing.assert_allclose(O, explicit_anchor_phase1(q, k, v, pos, b, a, apos, theta), rtol=0, atol=1e-12,
+                                   err_msg=name)
+        # the cache holds every token's own K/V, whatever the anchor
+        assert np.array_equal(ck, oracle.round_to_bf16(rope_complex(k, pos, theta))) and np.array_equal(cv, v)
+        rows = np.array([0, 5, 16, 17, 31, 32, 40, 47])
+        Or = oracle.phase1_rows(rows, q[rows], k, v, pos, b, theta, a, apos)
+        np.testing.assert_allclose(Or, O[rows], rtol=0, atol=1e-12, err_msg=name)
+
+
+def test_phase1_context_anchor_of_full_size_is_the_default():
+    """a = b with the anchor's own ids is the pages' default construction."""
+    theta = 500000.0
+    rng = np.random.default_rng(22)
+    L, b = 48, 16
+    q, k, v = _bf16_values(rng, (L, 4, 16)), _bf16_values(rng, (L, 2, 16)), _bf16_values(rng, (L, 2, 16))
+    pos = np.arange(L)
+    O0, _, _ = oracle.phase1(q, k, v, pos, b, theta)
+    O1, _, _ = oracle.phase1(q, k, v, pos, b, theta, b, np.tile(np.arange(b), (L // b - 1, 1)))
+    assert np.array_equal(O0, O1)
+    ref, _ = full_star_phase1(q, k, v, pos, b, theta)
+    np.testing.assert_allclose(O0, ref, rtol=0, atol=1e-12)
+
+
+def test_phase1_anchor_positions_are_relative():
+    """RoPE depends on position differences: shifting every position id (context and anchor) by
+    the same amount changes the outputs only through the bf16 rounding of the rotated values."""
+    theta = 500000.0
+    q, k, v, variants = _anchor_case(23)
+    L, b, a = q.shape[0], 16, 8
+    pos = np.arange(L)
+    for name, apos in variants.items():
+        O, _, _ = oracle.phase1(q, k, v, pos, b, theta, a, apos)
+        Os, _, _ = oracle.phase1(q, k, v, pos + 1000, b, theta, a, apos + 1000)
+        err = np.abs(O - Os)
+        assert err.max() < 2e-2 and err.mean() < 2e-3, (name, err.max(), err.mean())
+
+
+def test_planted_anchor_mistake_is_caught(monkeypatch):
+    """An oracle that ignores the anchor ids fails the explicit key-set pin for the offset and
+    zero-reset variants (and only for those)."""
+    theta = 500000.0
+    q, k, v, variants = _anchor_case(24)
+    L, b, a = q.shape[0], 16, 8
+    pos = np.arange(L)
+    real = oracle.augmented_context
+
+    def ignores_anchor_pos(L_, b_, pos_ctx=None, anchor=None, anchor_pos=None):
+        return real(L_, b_, pos_ctx, anchor, None)
+
+    monkeypatch.setattr(oracle.star_oracle, "augmented_context", ignores_anchor_pos)
+    for name, apos in variants.items():
+        O, _, _ = oracle.star_oracle.phase1(q, k, v, pos, b, theta, a, apos)
+        diff = np.abs(O - explicit_anchor_phase1(q, k, v, pos, b, a, apos, theta)).max()
+        if name == "context":
+            assert diff < 1e-12
+        else:
+            assert diff > 1e-2, (name, diff)
