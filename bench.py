@@ -130,12 +130,14 @@ class StarRun:
         self.star, self.wl, self.dev = star, wl, device
         self.inp = make_inputs(wl, device)
         self.shape = star.StarShape.make(B=wl.B, Hq=wl.Hq, Hkv=wl.Hkv, d=wl.d, L=wl.L, b=wl.b, T_max=wl.T_max,
-                                         page_tokens=wl.page_tokens, rope_theta=wl.theta)
+                                         page_tokens=wl.page_tokens, rope_theta=wl.theta, anchor=wl.anchor)
         self.cache = star.PagedKVCache(self.shape, device=device)
         self.o_ctx = torch.empty_like(self.inp["q_ctx"])
         self.o_part, self.lse_part = star.alloc_partials(self.shape, wl.T, device)
         self.ws2 = star.workspace(self.shape, star.STAR_OP_PHASE2, wl.T, device)
         self.wsd = star.workspace(self.shape, star.STAR_OP_DECODE, 0, device)
+        self.ws1 = (star.workspace(self.shape, star.STAR_OP_PHASE1_ANCHOR, 0, device)
+                    if "anchor_pos" in self.inp else None)
         self.o_q = torch.empty((wl.B, wl.T, wl.Hq, wl.d), dtype=torch.bfloat16, device=device)
         self.lse_q = torch.empty((wl.B, wl.T, wl.Hq), dtype=torch.float32, device=device)
         self.o_dec = torch.empty((wl.S, wl.B, 1, wl.Hq, wl.d), dtype=torch.bfloat16, device=device)
@@ -148,7 +150,12 @@ class StarRun:
         s, wl, inp = self.star, self.wl, self.inp
         if ev:
             s.star_set_trace_events(*ev["p1"])
-        s.star_phase1_encode(self.shape, self.cache, inp["q_ctx"], inp["k_ctx"], inp["v_ctx"], inp["pos_ctx"], self.o_ctx)
+        if self.ws1 is not None:
+            s.star_phase1_encode_anchored(self.shape, self.cache, inp["q_ctx"], inp["k_ctx"], inp["v_ctx"],
+                                          inp["pos_ctx"], inp["anchor_pos"], self.o_ctx, self.ws1)
+        else:
+            s.star_phase1_encode(self.shape, self.cache, inp["q_ctx"], inp["k_ctx"], inp["v_ctx"], inp["pos_ctx"],
+                                 self.o_ctx)
         if ev:
             s.star_set_trace_events(*ev["p2"])
         s.star_phase2_partial(self.shape, self.cache, inp["q_query"], inp["k_query"], inp["v_query"], inp["pos_query"],
@@ -300,7 +307,8 @@ def run_star(args, rank, world, local_rank):
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16; 1% of context key rows x8 where the workload says peaky)",
         "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d, "L": wl.L, "b": wl.b,
-                   "n": wl.n, "T": wl.T, "S": wl.S, "page_tokens": wl.page_tokens,
+                   "n": wl.n, "T": wl.T, "S": wl.S, "page_tokens": wl.page_tokens, "anchor": wl.a,
+                   "anchor_ids": wl.anchor_ids,
                    "parallelism": f"independent sequences per GPU x{world}",
                    "l2": "inputs larger than L2 (no flush)"},
         "phase1": {"attn_ms": p1_ms, "ctx_tok_s": wl.B * wl.L / (p1_ms * 1e-3), "tflops": tflops,
@@ -337,7 +345,7 @@ def run_e2e(run, K, W, world):
     import torch.distributed as dist
     wl, inp = run.wl, run.inp
     names = ["q_ctx", "k_ctx", "v_ctx", "pos_ctx", "q_query", "k_query", "v_query", "pos_query",
-             "q_dec", "k_dec", "v_dec", "pos_dec"]
+             "q_dec", "k_dec", "v_dec", "pos_dec"] + (["anchor_pos"] if "anchor_pos" in inp else [])
     out_names = ["o_ctx", "o_q", "lse_q", "o_dec", "lse_dec"]
     in_sets = [inp, {n: torch.empty_like(inp[n]) for n in names}]
     out_sets = [{n: getattr(run, n) for n in out_names}, {n: torch.empty_like(getattr(run, n)) for n in out_names}]
@@ -425,14 +433,16 @@ def oracle_phase1_sample(wl, host, blocks, rows_per_block, seed=0):
     v = host["v"].float().numpy().astype(np.float64)
     q = host["q"][rows].float().numpy().astype(np.float64)
     pos = host["pos"].numpy().astype(np.int64)
+    apos = host["anchor_pos"].numpy().astype(np.int64) if host.get("anchor_pos") is not None else None
     t = time.perf_counter()
-    oracle.phase1_rows(rows, q, k, v, pos, wl.b, wl.theta)
+    oracle.phase1_rows(rows, q, k, v, pos, wl.b, wl.theta, wl.anchor or None, apos)
     return len(rows), time.perf_counter() - t
 
 
 def _host_seq0(inp):
     return {"q": inp["q_ctx"][0].cpu(), "k": inp["k_ctx"][0].cpu(), "v": inp["v_ctx"][0].cpu(),
-            "pos": inp["pos_ctx"][0].cpu()}
+            "pos": inp["pos_ctx"][0].cpu(),
+            "anchor_pos": inp["anchor_pos"][0].cpu() if "anchor_pos" in inp else None}
 
 
 def cpu_baseline(run, rows_per_block):
@@ -467,7 +477,7 @@ def run_reference(args, rank, world):
         "warmup": W, "ms_per_step": 1e3 * tot_sec / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (same seeded inputs as the CUDA arm)",
         "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d, "L": wl.L, "b": wl.b,
-                   "n": wl.n, "T": wl.T, "S": wl.S},
+                   "n": wl.n, "T": wl.T, "S": wl.S, "anchor": wl.a, "anchor_ids": wl.anchor_ids},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
                          "sample": f"each step: float64 oracle Phase-1 output of {rows_per_block} context rows of one "
                                    f"block (all {wl.Hq} heads) of {wl.name}; value = rows/s"},

@@ -35,7 +35,7 @@ STAR_ERR_ALIGNMENT = -3
 STAR_ERR_CAPACITY = -4
 STAR_ERR_CUDA = -5
 STAR_ERR_TIMEOUT = -6
-STAR_OP_PHASE1, STAR_OP_PHASE2, STAR_OP_DECODE = 1, 2, 3
+STAR_OP_PHASE1, STAR_OP_PHASE2, STAR_OP_DECODE, STAR_OP_PHASE1_ANCHOR = 1, 2, 3, 4
 
 
 class StarError(RuntimeError):
@@ -48,12 +48,13 @@ class StarShape(ctypes.Structure):
     _fields_ = [
         ("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("d", ctypes.c_int32),
         ("L", ctypes.c_int32), ("b", ctypes.c_int32), ("n", ctypes.c_int32), ("T_max", ctypes.c_int32),
-        ("page_tokens", ctypes.c_int32), ("rope_theta", ctypes.c_double),
+        ("page_tokens", ctypes.c_int32), ("rope_theta", ctypes.c_double), ("anchor", ctypes.c_int32),
     ]
 
     @classmethod
-    def make(cls, B, Hq, Hkv, d, L, b, T_max, page_tokens=256, rope_theta=500000.0) -> "StarShape":
-        return cls(B, Hq, Hkv, d, L, b, L // b if b else 0, T_max, page_tokens, rope_theta)
+    def make(cls, B, Hq, Hkv, d, L, b, T_max, page_tokens=256, rope_theta=500000.0, anchor=0) -> "StarShape":
+        """anchor: the anchor size a (the first a tokens of block 1); 0 means b."""
+        return cls(B, Hq, Hkv, d, L, b, L // b if b else 0, T_max, page_tokens, rope_theta, anchor)
 
 
 class StarCache(ctypes.Structure):
@@ -83,6 +84,7 @@ def lib() -> ctypes.CDLL:
             "star_build_positions": ([P(StarShape), P(StarCache), V, V, V, V], ctypes.c_int),
             "star_kv_append": ([P(StarShape), P(StarCache), V, V, V, I32, I32, V], ctypes.c_int),
             "star_phase1_encode": ([P(StarShape), P(StarCache), V, V, V, V, V, V, SZ, V], ctypes.c_int),
+            "star_phase1_encode_anchored": ([P(StarShape), P(StarCache), V, V, V, V, V, V, V, SZ, V], ctypes.c_int),
             "star_phase2_partial": ([P(StarShape), P(StarCache), V, V, V, V, I32, V, V, V, SZ, V], ctypes.c_int),
             "star_lse_merge": ([I32, I64, I32, V, V, V, V, V], ctypes.c_int),
             "star_decode_step": ([P(StarShape), P(StarCache), V, V, V, V, I32, V, V, V, SZ, V], ctypes.c_int),
@@ -203,6 +205,16 @@ def star_phase1_encode(shape, cache: PagedKVCache, q, k, v, pos_ctx, out, ws=Non
                                     _ptr(pos_ctx, "pos_ctx", torch.int32), _ptr(out, "out", torch.bfloat16),
                                     _ptr(ws, "ws"), 0 if ws is None else ws.numel() * ws.element_size(),
                                     _stream(stream)))
+
+
+def star_phase1_encode_anchored(shape, cache: PagedKVCache, q, k, v, pos_ctx, anchor_pos, out, ws=None, stream=None):
+    """Phase 1 with the anchor's position ids per block (int32 [B][n-1][a], or None for the default)."""
+    _check(lib().star_phase1_encode_anchored(ctypes.byref(shape), ctypes.byref(cache.c), _ptr(q, "q", torch.bfloat16),
+                                             _ptr(k, "k", torch.bfloat16), _ptr(v, "v", torch.bfloat16),
+                                             _ptr(pos_ctx, "pos_ctx", torch.int32),
+                                             _ptr(anchor_pos, "anchor_pos", torch.int32),
+                                             _ptr(out, "out", torch.bfloat16), _ptr(ws, "ws"),
+                                             0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def star_phase2_partial(shape, cache: PagedKVCache, q, k, v, q_pos, T: int, o_part, lse_part, ws=None, stream=None):

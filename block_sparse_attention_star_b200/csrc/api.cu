@@ -68,6 +68,10 @@ int check_shape(const star_shape* s) {
   if (s->page_tokens % 128) return fail(STAR_ERR_UNSUPPORTED_SHAPE, "page_tokens (%d) must be a multiple of 128", s->page_tokens);
   if (s->b % s->page_tokens)
     return fail(STAR_ERR_UNSUPPORTED_SHAPE, "b (%d) must be a multiple of page_tokens (%d)", s->b, s->page_tokens);
+  if (s->anchor < 0) return fail(STAR_ERR_INVALID_ARG, "anchor size (%d) must not be negative", s->anchor);
+  if (s->anchor > s->b || s->anchor % 128)
+    return fail(STAR_ERR_UNSUPPORTED_SHAPE, "anchor size (%d) must be a multiple of 128 and at most b (%d)", s->anchor,
+                s->b);
   if ((int64_t)s->L + round_up(s->T_max, 128) >= (int64_t)1 << 30)
     return fail(STAR_ERR_UNSUPPORTED_SHAPE, "L + T_max too large");
   return STAR_OK;
@@ -150,6 +154,13 @@ size_t phase2_ws_bytes(const star_shape* s, int T) {
   return round_up(parts * rows * s->d * sizeof(float), 256) + round_up(parts * rows * sizeof(float), 256);
 }
 
+int anchor_of(const star_shape* s) { return s->anchor ? s->anchor : s->b; }
+
+// The anchor's keys, roped at caller-given ids, per (sequence, block 2..n): bf16 [B][n-1][Hkv][a][d].
+size_t anchor_ws_bytes(const star_shape* s) {
+  return (size_t)s->B * (s->n - 1) * s->Hkv * anchor_of(s) * s->d * 2;
+}
+
 int decode_chunk(const star_shape* s) {
   return star::decode_pick_chunk(s->B, s->Hkv, s->Hq / s->Hkv, s->L + s->T_max, num_sms());
 }
@@ -204,6 +215,7 @@ int star_workspace_size(const star_shape* shape, int op, int32_t T, size_t* byte
       *bytes_out = phase2_ws_bytes(shape, T);
       return STAR_OK;
     case STAR_OP_DECODE: *bytes_out = decode_ws_bytes(shape); return STAR_OK;
+    case STAR_OP_PHASE1_ANCHOR: *bytes_out = anchor_ws_bytes(shape); return STAR_OK;
     default: return fail(STAR_ERR_INVALID_ARG, "unknown op %d", op);
   }
 }
@@ -216,7 +228,8 @@ int star_build_positions(const star_shape* shape, const star_cache* cache, const
   STAR_REQUIRE_PTR4(pos_ctx, "pos_ctx");
   STAR_REQUIRE_PTR4(aug_pos, "aug_pos");
   STAR_REQUIRE_PTR4(block_map, "block_map");
-  cudaError_t e = star::launch_build_positions(pos_ctx, shape->B, shape->L, shape->b, view(shape, cache), aug_pos,
+  cudaError_t e = star::launch_build_positions(pos_ctx, shape->B, shape->L, shape->b, anchor_of(shape),
+                                               view(shape, cache), aug_pos,
                                                block_map, (cudaStream_t)stream);
   return e == cudaSuccess ? STAR_OK : cuda_fail(e, "build_positions launch");
 }
@@ -239,8 +252,12 @@ int star_kv_append(const star_shape* shape, const star_cache* cache, const void*
 
 int star_phase1_encode(const star_shape* shape, const star_cache* cache, const void* q, const void* k, const void* v,
                        const int32_t* pos_ctx, void* out, void* ws, size_t ws_bytes, star_stream_t stream) {
-  (void)ws;
-  (void)ws_bytes;
+  return star_phase1_encode_anchored(shape, cache, q, k, v, pos_ctx, nullptr, out, ws, ws_bytes, stream);
+}
+
+int star_phase1_encode_anchored(const star_shape* shape, const star_cache* cache, const void* q, const void* k,
+                                const void* v, const int32_t* pos_ctx, const int32_t* anchor_pos, void* out,
+                                void* ws, size_t ws_bytes, star_stream_t stream) {
   int rc = check_shape(shape);
   if (!rc) rc = check_cache(shape, cache);
   if (rc) return rc;
@@ -249,6 +266,13 @@ int star_phase1_encode(const star_shape* shape, const star_cache* cache, const v
   STAR_REQUIRE_PTR(v, "v");
   STAR_REQUIRE_PTR4(pos_ctx, "pos_ctx");
   STAR_REQUIRE_PTR(out, "out");
+  if (anchor_pos && shape->n > 1) {
+    STAR_REQUIRE_PTR4(anchor_pos, "anchor_pos");
+    STAR_REQUIRE_PTR(ws, "ws");
+    const size_t need = anchor_ws_bytes(shape);
+    if (ws_bytes < need)
+      return fail(STAR_ERR_CAPACITY, "workspace %zu bytes < %zu needed for the anchor's keys", ws_bytes, need);
+  }
   cudaStream_t st = (cudaStream_t)stream;
   const star::CacheView cv = view(shape, cache);
   const star::RopeTable rt = rope_table(shape);
@@ -257,9 +281,17 @@ int star_phase1_encode(const star_shape* shape, const star_cache* cache, const v
   e = star::launch_zero_slots(shape->B, shape->L, shape->L + (int)round_up(shape->T_max, 128), shape->Hkv, shape->d,
                               cv, st);
   if (e != cudaSuccess) return cuda_fail(e, "phase1 tail clear");
+  const int anchor = anchor_of(shape);
+  const bool own_anchor_ids = anchor_pos && shape->n > 1;
+  if (own_anchor_ids) {
+    e = star::launch_rope_anchor(k, anchor_pos, shape->B, shape->L, shape->n, anchor, shape->Hkv, shape->d, ws, rt, st);
+    if (e != cudaSuccess) return cuda_fail(e, "phase1 anchor keys");
+  }
   star::AttnLaunch a;
   memset(&a, 0, sizeof(a));
   a.mode = 0;
+  a.anchor = anchor;
+  a.anchor_k = own_anchor_ids ? ws : nullptr;
   a.B = shape->B;
   a.Hq = shape->Hq;
   a.Hkv = shape->Hkv;

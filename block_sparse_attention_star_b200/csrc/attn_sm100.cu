@@ -72,6 +72,8 @@ struct Params {
   // Phase-2 tiling
   int chunk_keys, chunks_per_block, tail_tiles, TQ, HT, NTT, NHT, npairs;
   int num_items;
+  // Phase-1 anchor: its size, and whether its keys come from the tmKA map (roped at caller ids)
+  int anchor, anchor_k_on;
   float scale_log2;
   double inv_freq[kMaxHalfDim];
 };
@@ -114,7 +116,7 @@ __device__ __forceinline__ Item decode_item(const Params& p, int idx) {
       it.hp = w - (w / npairs) * npairs;
     }
     it.a_start = 0;
-    it.a_tiles = (i > 0) ? nqt : 0;
+    it.a_tiles = (i > 0) ? p.anchor / kRows : 0;  // the anchor: the first a keys of block 1
     it.b_start = i * p.b;
     it.b_tiles = t + 1;
     it.part = i;
@@ -224,7 +226,8 @@ struct Smem {
 template <int D, int MODE, int NSK, int NSV>
 __global__ void __launch_bounds__(kThreads, 1)
     star_attn_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ Params p) {
+                     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKA,
+                     const __grid_constant__ Params p) {
   using S = Smem<D, MODE, NSK, NSV>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -264,6 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
     if (MODE == 0) prefetch_tmap(&tmQ);
+    if (MODE == 0 && p.anchor_k_on) prefetch_tmap(&tmKA);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -297,9 +301,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             mbar_arrive_expect_tx(&k_full[s], S::kTile);
             uint8_t* dst = smem + S::kK + s * S::kTile;
+            if (MODE == 0 && p.anchor_k_on && j < it.a_tiles) {
+              // The anchor's keys roped at the caller's ids: [B][n-1][Hkv][a][d], block it.part.
 #pragma unroll
-            for (int h = 0; h < D / 64; ++h)
-              tma_load_4d(dst + h * (kKeys * 128), &tmK, &k_full[s], h * 64, slot, it.g, page);
+              for (int h = 0; h < D / 64; ++h)
+                tma_load_4d(dst + h * (kKeys * 128), &tmKA, &k_full[s], h * 64, j * kKeys, it.g,
+                            it.bi * (p.n - 1) + it.part - 1);
+            } else {
+#pragma unroll
+              for (int h = 0; h < D / 64; ++h)
+                tma_load_4d(dst + h * (kKeys * 128), &tmK, &k_full[s], h * 64, slot, it.g, page);
+            }
             ++kcnt;
           }
           {
@@ -678,6 +690,20 @@ bool make_q_map(CUtensorMap* map, const void* q, int d, int Hq, int L, int B) {
   return r == CUDA_SUCCESS;
 }
 
+// The anchor's keys [B*(n-1)][Hkv][a][d] bf16 as a 4-D tensor (d innermost); box = 64 x 128 keys x 1 x 1.
+bool make_anchor_map(CUtensorMap* map, const void* ka, int d, int a, int Hkv, int nseq) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)a, (cuuint64_t)Hkv, (cuuint64_t)nseq};
+  const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)a * d * 2, (cuuint64_t)Hkv * a * d * 2};
+  const cuuint32_t box[4] = {64, (cuuint32_t)kKeys, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ka), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int pow2_at_least(int x) {
   int v = 1;
   while (v < x) v <<= 1;
@@ -686,7 +712,7 @@ int pow2_at_least(int x) {
 
 template <int D, int MODE>
 cudaError_t launch_typed(const AttnLaunch& a, const Params& p, const CUtensorMap& mk, const CUtensorMap& mv,
-                         const CUtensorMap& mq, cudaStream_t st) {
+                         const CUtensorMap& mq, const CUtensorMap& mka, cudaStream_t st) {
   constexpr int NSK = (D == 128) ? 2 : 4;
   constexpr int NSV = (D == 128) ? 2 : 4;
   using S = Smem<D, MODE, NSK, NSV>;
@@ -702,7 +728,7 @@ cudaError_t launch_typed(const AttnLaunch& a, const Params& p, const CUtensorMap
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = std::min(p.num_items, sms);
   if (grid <= 0) return cudaSuccess;
-  kern<<<grid, kThreads, S::kBytes, st>>>(mk, mv, mq, p);
+  kern<<<grid, kThreads, S::kBytes, st>>>(mk, mv, mq, mka, p);
   return cudaGetLastError();
 }
 
@@ -756,10 +782,17 @@ cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t st, const char** 
     if (why) *why = "cuTensorMapEncodeTiled failed for the rotated queries";
     return cudaErrorInvalidValue;
   }
+  CUtensorMap mka = mk;  // unused unless the anchor's keys are roped at caller ids
+  p.anchor = a.mode == 0 ? a.anchor : 0;
+  p.anchor_k_on = (a.mode == 0 && a.anchor_k && a.n > 1) ? 1 : 0;
+  if (p.anchor_k_on && !make_anchor_map(&mka, a.anchor_k, a.d, a.anchor, a.Hkv, a.B * (a.n - 1))) {
+    if (why) *why = "cuTensorMapEncodeTiled failed for the anchor's keys";
+    return cudaErrorInvalidValue;
+  }
   if (a.d == 128) {
-    return a.mode == 0 ? launch_typed<128, 0>(a, p, mk, mv, mq, st) : launch_typed<128, 1>(a, p, mk, mv, mq, st);
+    return a.mode == 0 ? launch_typed<128, 0>(a, p, mk, mv, mq, mka, st) : launch_typed<128, 1>(a, p, mk, mv, mq, mka, st);
   } else {
-    return a.mode == 0 ? launch_typed<64, 0>(a, p, mk, mv, mq, st) : launch_typed<64, 1>(a, p, mk, mv, mq, st);
+    return a.mode == 0 ? launch_typed<64, 0>(a, p, mk, mv, mq, mka, st) : launch_typed<64, 1>(a, p, mk, mv, mq, mka, st);
   }
 }
 

@@ -34,9 +34,13 @@ cudaError_t launch_rope_q(const void* q, const int32_t* pos, int B, int ntok, in
                           const RopeTable& rt, cudaStream_t st);
 // Zero cache slots [from, to) of every sequence (K and V).
 cudaError_t launch_zero_slots(int B, int from, int to, int Hkv, int d, const CacheView& c, cudaStream_t st);
-// c' position ids [B][L + (n-1) b] and block map [B][L][3].
-cudaError_t launch_build_positions(const int32_t* pos_ctx, int B, int L, int b, const CacheView& c,
+// c' position ids [B][L + (n-1) a] (anchor = the first a tokens) and block map [B][L][3].
+cudaError_t launch_build_positions(const int32_t* pos_ctx, int B, int L, int b, int a, const CacheView& c,
                                    int32_t* aug_pos, int32_t* block_map, cudaStream_t st);
+// The anchor's keys roped at caller ids: out[bi][i-1][h][j] = RoPE(k[bi][j][h], anchor_pos[bi][i-1][j])
+// for blocks i = 1..n-1 (0-based), j < a.  k: [B][L][Hkv][d] bf16; out: bf16 [B][n-1][Hkv][a][d].
+cudaError_t launch_rope_anchor(const void* k, const int32_t* anchor_pos, int B, int L, int n, int a, int Hkv, int d,
+                               void* out, const RopeTable& rt, cudaStream_t st);
 
 // --- merge.cu ---------------------------------------------------------------
 // groups x rows outputs; group g merges input parts [g*parts_per_group, (g+1)*parts_per_group).
@@ -56,6 +60,8 @@ struct AttnLaunch {
   float* out_f32;         // mode 1: [parts][B][T][Hq][d]
   float* lse_f32;         // mode 1: [parts][B][T][Hq]
   int chunks_per_block;   // mode 1
+  int anchor;             // mode 0: anchor size a (the first a keys of block 1)
+  const void* anchor_k;   // mode 0: NULL (anchor keys are block 1's cached keys) or bf16 [B][n-1][Hkv][a][d]
   float scale_log2;
   RopeTable rope;
 };

@@ -12,6 +12,7 @@
 //   0 * V must stay 0).
 // * rope_q: the query heads rotated by RoPE once, before the attention kernel
 //   (which then stages Q tiles by TMA instead of rotating them per work item).
+// * rope_anchor: the anchor's keys roped at caller-given ids (anchor variants).
 // * build_positions: the integer position ids of c' and the token -> (block,
 //   page, slot) map ("被增广的上下文").
 //
@@ -113,6 +114,44 @@ __global__ void __launch_bounds__(256) rope_q_kernel(const bf16* q, const int32_
   }
 }
 
+// The anchor's keys roped at caller ids, one thread per (sequence, block, anchor token,
+// 8-pair chunk): out[bi][i-1][h][j] = RoPE(k[bi][j][h], anchor_pos[bi][i-1][j]) for every KV head.
+template <int D>
+__global__ void __launch_bounds__(256) rope_anchor_kernel(const bf16* __restrict__ k, const int32_t* __restrict__ apos,
+                                                          int B, int L, int nb, int a, int Hkv, bf16* __restrict__ out,
+                                                          const __grid_constant__ RopeParams rp) {
+  constexpr int CH = D / 16;
+  const long long total = (long long)B * nb * a * CH;
+  for (long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x; gid < total;
+       gid += (long long)gridDim.x * blockDim.x) {
+    const int c = (int)(gid % CH);
+    long long r = gid / CH;
+    const int j = (int)(r % a);
+    r /= a;  // bi * nb + block
+    const int bi = (int)(r / nb);
+    const int p_t = apos[r * a + j];
+    double cs[4][2], sn[4][2];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      rope_sincos(p_t, rp.inv_freq[8 * c + 2 * e], cs[e][0], sn[e][0]);
+      rope_sincos(p_t, rp.inv_freq[8 * c + 2 * e + 1], cs[e][1], sn[e][1]);
+    }
+    for (int h = 0; h < Hkv; ++h) {
+      const size_t src = (((size_t)bi * L + j) * Hkv + h) * D;
+      const size_t dst = ((size_t)(r * Hkv + h) * a + j) * D;
+      const uint4 x = __ldg(reinterpret_cast<const uint4*>(k + src + 8 * c));
+      const uint4 y = __ldg(reinterpret_cast<const uint4*>(k + src + D / 2 + 8 * c));
+      const uint32_t* xw = reinterpret_cast<const uint32_t*>(&x);
+      const uint32_t* yw = reinterpret_cast<const uint32_t*>(&y);
+      uint32_t lo[4], hi[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) rope_rotate2(xw[e], yw[e], cs[e], sn[e], lo[e], hi[e]);
+      *reinterpret_cast<uint4*>(out + dst + 8 * c) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      *reinterpret_cast<uint4*>(out + dst + D / 2 + 8 * c) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    }
+  }
+}
+
 __global__ void zero_slots_kernel(int B, int from, int to, int Hkv, int d, bf16* kpool, bf16* vpool,
                                   const int32_t* page_table, int max_pages, int num_pages, int P) {
   const int CH = d / 8;
@@ -137,24 +176,25 @@ __global__ void zero_slots_kernel(int B, int from, int to, int Hkv, int d, bf16*
   }
 }
 
-// Augmented row a of sequence bi: block 0 holds rows [0, b); block i >= 1 holds
-// rows [b + 2b(i-1), b + 2b i): b anchor rows (ids of tokens 0..b-1) then its own.
-__global__ void build_positions_kernel(const int32_t* pos_ctx, int B, int L, int b, const int32_t* page_table,
-                                       int max_pages, int P, int32_t* aug_pos, int32_t* block_map) {
+// Augmented row r of sequence bi: block 0 holds rows [0, b); block i >= 1 holds
+// rows [b + (a+b)(i-1), b + (a+b) i): the a anchor rows (ids of tokens 0..a-1) then its own.
+__global__ void build_positions_kernel(const int32_t* pos_ctx, int B, int L, int b, int anc,
+                                       const int32_t* page_table, int max_pages, int P, int32_t* aug_pos,
+                                       int32_t* block_map) {
   const int n = L / b;
-  const long long aug_len = (long long)L + (long long)(n - 1) * b;
+  const long long aug_len = (long long)L + (long long)(n - 1) * anc;
   const long long total = (long long)B * aug_len;
   for (long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x; gid < total;
        gid += (long long)gridDim.x * blockDim.x) {
     const int bi = (int)(gid / aug_len);
-    const long long a = gid % aug_len;
+    const long long r = gid % aug_len;
     long long tok;
-    if (a < b) {
-      tok = a;
+    if (r < b) {
+      tok = r;
     } else {
-      const long long i = 1 + (a - b) / (2LL * b);
-      const long long off = (a - b) % (2LL * b);
-      tok = off < b ? off : i * b + (off - b);
+      const long long i = 1 + (r - b) / ((long long)anc + b);
+      const long long off = (r - b) % ((long long)anc + b);
+      tok = off < anc ? off : i * b + (off - anc);
     }
     aug_pos[gid] = pos_ctx[(size_t)bi * L + tok];
   }
@@ -226,11 +266,27 @@ cudaError_t launch_zero_slots(int B, int from, int to, int Hkv, int d, const Cac
   return cudaGetLastError();
 }
 
-cudaError_t launch_build_positions(const int32_t* pos_ctx, int B, int L, int b, const CacheView& c, int32_t* aug_pos,
-                                   int32_t* block_map, cudaStream_t st) {
-  const long long work = (long long)B * (L + (long long)(L / b - 1) * b);
-  build_positions_kernel<<<grid_for(work, 256), 256, 0, st>>>(pos_ctx, B, L, b, c.page_table, c.max_pages, c.P,
+cudaError_t launch_build_positions(const int32_t* pos_ctx, int B, int L, int b, int a, const CacheView& c,
+                                   int32_t* aug_pos, int32_t* block_map, cudaStream_t st) {
+  const long long work = (long long)B * (L + (long long)(L / b - 1) * a);
+  build_positions_kernel<<<grid_for(work, 256), 256, 0, st>>>(pos_ctx, B, L, b, a, c.page_table, c.max_pages, c.P,
                                                                aug_pos, block_map);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope_anchor(const void* k, const int32_t* anchor_pos, int B, int L, int n, int a, int Hkv, int d,
+                               void* out, const RopeTable& rt, cudaStream_t st) {
+  if (n <= 1 || a <= 0) return cudaSuccess;
+  RopeParams rp;
+  for (int j = 0; j < d / 2; ++j) rp.inv_freq[j] = rt.inv_freq[j];
+  const long long work = (long long)B * (n - 1) * a * (d / 16);
+  const int grid = grid_for(work, 256);
+  if (d == 128)
+    rope_anchor_kernel<128><<<grid, 256, 0, st>>>(reinterpret_cast<const bf16*>(k), anchor_pos, B, L, n - 1, a, Hkv,
+                                                  reinterpret_cast<bf16*>(out), rp);
+  else
+    rope_anchor_kernel<64><<<grid, 256, 0, st>>>(reinterpret_cast<const bf16*>(k), anchor_pos, B, L, n - 1, a, Hkv,
+                                                 reinterpret_cast<bf16*>(out), rp);
   return cudaGetLastError();
 }
 

@@ -55,7 +55,7 @@ enum {
 };
 
 /* Workspace query selectors. */
-enum { STAR_OP_PHASE1 = 1, STAR_OP_PHASE2 = 2, STAR_OP_DECODE = 3 };
+enum { STAR_OP_PHASE1 = 1, STAR_OP_PHASE2 = 2, STAR_OP_DECODE = 3, STAR_OP_PHASE1_ANCHOR = 4 };
 
 /* Problem shape ("问题定义与记号": context c of n blocks of b tokens, query q). */
 typedef struct star_shape {
@@ -64,11 +64,14 @@ typedef struct star_shape {
   int32_t Hkv;         /* key/value heads */
   int32_t d;           /* head dim: 64 or 128 */
   int32_t L;           /* context tokens, L = n * b */
-  int32_t b;           /* block size (anchor size = b); multiple of 128 and of page_tokens */
+  int32_t b;           /* block size; multiple of 128 and of page_tokens */
   int32_t n;           /* number of blocks */
   int32_t T_max;       /* tail capacity after the context: query + generated tokens */
   int32_t page_tokens; /* P: tokens per cache page; multiple of 128 */
   double rope_theta;   /* RoPE base, e.g. 500000 */
+  int32_t anchor;      /* anchor size a: the first a tokens of block 1 ("仓库里的真实实现":
+                          anchor_block_size is a parameter of its own); 0 means b (the pages'
+                          default, the whole first block); a multiple of 128 and <= b */
 } star_shape;
 
 /* Paged KV cache ("局部注意力与 KV 丢弃": only non-anchor KV is kept).
@@ -102,13 +105,16 @@ int star_pages_needed(const star_shape* shape, int32_t* max_pages_out);
 int star_page_table_fill(const star_shape* shape, int32_t* page_table_host, int32_t max_pages, int32_t first_page);
 
 /* Bytes of scratch the given operation needs (op = STAR_OP_*; for STAR_OP_PHASE2
- * T is the number of query tokens of the call, ignored otherwise). */
+ * T is the number of query tokens of the call, ignored otherwise).
+ * STAR_OP_PHASE1: 0.  STAR_OP_PHASE1_ANCHOR: star_phase1_encode_anchored with anchor
+ * position ids, B*(n-1)*Hkv*a*d*2 bytes (the anchor's keys roped at those ids). */
 int star_workspace_size(const star_shape* shape, int op, int32_t T, size_t* bytes_out);
 
 /* Integer structure of c' ("被增广的上下文"), for checking only.
  * pos_ctx:   device int32 [B][L], position id of each context token (normally t).
- * aug_pos:   device int32 [B][L + (n-1)*b], position ids of c' = [c_1, (c_1 c_2), ...,
- *            (c_1 c_n)]: block 1 then, per block i>1, b anchor ids then c_i's ids.
+ * aug_pos:   device int32 [B][L + (n-1)*a], position ids of c' = [c_1, (a_1 c_2), ...,
+ *            (a_1 c_n)] with a_1 the anchor (the first a = shape->anchor tokens of c_1, a = b
+ *            by default): block 1 then, per block i>1, the a anchor ids then c_i's ids.
  * block_map: device int32 [B][L][3]: (block t/b, physical page, slot t % page_tokens).
  * Errors: INVALID_ARG, UNSUPPORTED_SHAPE (L != n*b), CAPACITY, CUDA. */
 int star_build_positions(const star_shape* shape, const star_cache* cache, const int32_t* pos_ctx,
@@ -126,8 +132,8 @@ int star_kv_append(const star_shape* shape, const star_cache* cache, const void*
  * ("Phase 1: 被增广的上下文", "局部注意力与 KV 丢弃", "复杂度分析").
  * q: bf16 [B][L][Hq][d]; k, v: bf16 [B][L][Hkv][d]; pos_ctx: device int32 [B][L].
  * Writes out: bf16 [B][L][Hq][d], where row t of block i attends to the anchor
- * keys [0, b) (for i > 1) and to its own block's keys up to t, each key roped at
- * its own position id.  Writes RoPE(K), V of the L context tokens into cache
+ * keys [0, a) (for i > 1; a = shape->anchor, b by default) and to its own block's keys
+ * up to t, each key roped at its own position id.  Writes RoPE(K), V of the L context tokens into cache
  * slots [0, L) (the anchor copies are never written) and zeroes slots
  * [L, L + round_up(T_max,128)).  out also serves as the staging buffer of RoPE(q)
  * during the call (each row is rotated there, then overwritten by its output), so
@@ -136,6 +142,20 @@ int star_kv_append(const star_shape* shape, const star_cache* cache, const void*
 int star_phase1_encode(const star_shape* shape, const star_cache* cache, const void* q, const void* k,
                        const void* v, const int32_t* pos_ctx, void* out, void* ws, size_t ws_bytes,
                        star_stream_t stream);
+
+/* Phase 1 with the anchor's position ids given per block (the anchor variants of
+ * "仓库里的真实实现" and the implementers' notes on that page: the anchor's ids may be
+ * sampled from the prefix range, or reset to 0, instead of keeping tokens 0..a-1's ids).
+ * anchor_pos: device int32 [B][n-1][a]; row i-2 holds the ids of the anchor's a tokens in
+ * block i (2 <= i <= n).  NULL: the anchor keeps the ids of tokens 0..a-1 (pos_ctx), exactly
+ * star_phase1_encode.  Otherwise the anchor's keys RoPE(k_j, anchor_pos[..][j]) are
+ * written into ws (bf16 [B][n-1][Hkv][a][d], star_workspace_size(STAR_OP_PHASE1_ANCHOR))
+ * and read from there; the anchor's values are block 1's cached values (V has no
+ * position).  The cache contents are the same as star_phase1_encode's.
+ * Errors: as star_phase1_encode; CAPACITY if ws_bytes is too small. */
+int star_phase1_encode_anchored(const star_shape* shape, const star_cache* cache, const void* q, const void* k,
+                                const void* v, const int32_t* pos_ctx, const int32_t* anchor_pos, void* out,
+                                void* ws, size_t ws_bytes, star_stream_t stream);
 
 /* Phase 2 per-block partials ("Phase 2: 局部注意力与本地统计量": A_h and s_h per host).
  * q: bf16 [B][T][Hq][d]; k, v: bf16 [B][T][Hkv][d] or both NULL (already appended);

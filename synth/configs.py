@@ -31,6 +31,13 @@ class Workload:
     theta: float = 500000.0
     seed: int = 0
     page_tokens: int = 256
+    anchor: int = 0                 # anchor size a (the first a tokens of block 1); 0 = b
+    anchor_ids: str = "context"     # anchor position ids: "context" (tokens 0..a-1's own),
+                                    # "offset" (per block, a seeded offset inside the prefix), "zero"
+
+    @property
+    def a(self) -> int:
+        return self.anchor or self.b
 
     @property
     def n(self) -> int:
@@ -56,12 +63,12 @@ class Workload:
         """(query row, key) pairs Phase 1 computes for one head of one sequence.
 
         Block 1 is plain causal (b(b+1)/2 pairs); every later block sees the
-        whole anchor (b*b) plus its own causal triangle.  Anchor rows are not
+        whole anchor (a*b) plus its own causal triangle.  Anchor rows are not
         recomputed, so they are not counted.
         """
-        b, n = self.b, self.n
+        b, n, a = self.b, self.n, self.a
         tri = b * (b + 1) // 2
-        return tri + (n - 1) * (b * b + tri)
+        return tri + (n - 1) * (a * b + tri)
 
     def phase1_flops(self) -> float:
         return 4.0 * self.d * self.Hq * self.B * self.phase1_pairs_per_head()
@@ -88,6 +95,11 @@ CONFIGS: dict[str, Workload] = {
     "llama8b-128k-b4096": _BASE["llama8b-128k"].with_block(4096),
     "llama70b-128k": _BASE["llama70b-128k"],
     "ctx-1m": _BASE["ctx-1m"],
+    # anchor variants: a quarter-block anchor with per-block offset ids, a zero-reset anchor
+    "llama8b-128k-b32768-a8192-offset": dataclasses.replace(_BASE["llama8b-128k"], name="llama8b-128k-b32768-a8192-offset",
+                                                            anchor=8192, anchor_ids="offset"),
+    "llama8b-128k-b32768-zero": dataclasses.replace(_BASE["llama8b-128k"], name="llama8b-128k-b32768-zero",
+                                                    anchor_ids="zero"),
 }
 
 

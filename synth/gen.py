@@ -42,6 +42,7 @@ STREAM_IDS = {
     "q_query": 4, "k_query": 5, "v_query": 6,
     "q_dec": 7, "k_dec": 8, "v_dec": 9,
     "peaky": 10,
+    "anchor": 11,
 }
 
 _CHUNK = 1 << 24
@@ -138,6 +139,24 @@ def peaky_rows(wl: Workload, device="cpu") -> torch.Tensor:
     return torch.stack(rows)
 
 
+def anchor_positions(wl: Workload, device="cpu") -> torch.Tensor:
+    """The anchor's position ids per (sequence, block i >= 1), int32 [B, n-1, a].
+
+    "zero": every id 0.  "offset": ids o + 0..a-1 with o drawn uniformly (seeded) from
+    [0, i*b - a], i.e. the anchor placed inside the prefix that precedes block i."""
+    B, n, b, a = wl.B, wl.n, wl.b, wl.a
+    if wl.anchor_ids == "zero":
+        return torch.zeros((B, n - 1, a), dtype=torch.int32, device=device)
+    if wl.anchor_ids != "offset":
+        raise ValueError(f"unknown anchor ids {wl.anchor_ids!r}")
+    key = stream_key(wl.seed, STREAM_IDS["anchor"])
+    idx = torch.arange(B * (n - 1), dtype=torch.int64, device=device)
+    u = counter_u64(key, idx) & ((1 << 62) - 1)
+    span = (idx % (n - 1) + 1) * b - a + 1          # block i = idx % (n-1) + 1
+    off = (u % span).view(B, n - 1, 1)
+    return (off + torch.arange(a, dtype=torch.int64, device=device)).to(torch.int32).contiguous()
+
+
 def make_inputs(wl: Workload, device="cpu", parts=("ctx", "query", "dec")) -> dict[str, torch.Tensor]:
     """All inputs of one workload (bf16 values, int32 positions)."""
     B, L, T, S, Hq, Hkv, d = wl.B, wl.L, wl.T, wl.S, wl.Hq, wl.Hkv, wl.d
@@ -152,6 +171,8 @@ def make_inputs(wl: Workload, device="cpu", parts=("ctx", "query", "dec")) -> di
                 for h in range(Hkv):
                     g["k_ctx"][bi, rows[bi, h], h, :] *= 8
         g["pos_ctx"] = torch.arange(L, dtype=torch.int32, device=device).repeat(B, 1).contiguous()
+        if wl.anchor_ids != "context" and wl.n > 1:
+            g["anchor_pos"] = anchor_positions(wl, device)
     if "query" in parts:
         g["q_query"] = gaussian_bf16(wl.seed, STREAM_IDS["q_query"], (B, T, Hq, d), device)
         g["k_query"] = gaussian_bf16(wl.seed, STREAM_IDS["k_query"], (B, T, Hkv, d), device)

@@ -23,7 +23,7 @@ LSE_ABS = 1e-3
 
 def shape_of(wl: Workload) -> star.StarShape:
     return star.StarShape.make(B=wl.B, Hq=wl.Hq, Hkv=wl.Hkv, d=wl.d, L=wl.L, b=wl.b, T_max=wl.T_max,
-                               page_tokens=wl.page_tokens, rope_theta=wl.theta)
+                               page_tokens=wl.page_tokens, rope_theta=wl.theta, anchor=wl.anchor)
 
 
 def to64(t: torch.Tensor) -> np.ndarray:
@@ -39,7 +39,12 @@ def run_gpu(wl: Workload, inp: dict, page_table: torch.Tensor | None = None, num
     res = {"cache": cache, "shape": shape}
     if "phase1" in phases:
         out = torch.empty_like(inp["q_ctx"])
-        star.star_phase1_encode(shape, cache, inp["q_ctx"], inp["k_ctx"], inp["v_ctx"], inp["pos_ctx"], out)
+        if inp.get("anchor_pos") is not None:
+            ws1 = star.workspace(shape, star.STAR_OP_PHASE1_ANCHOR, 0, dev)
+            star.star_phase1_encode_anchored(shape, cache, inp["q_ctx"], inp["k_ctx"], inp["v_ctx"], inp["pos_ctx"],
+                                             inp["anchor_pos"], out, ws1)
+        else:
+            star.star_phase1_encode(shape, cache, inp["q_ctx"], inp["k_ctx"], inp["v_ctx"], inp["pos_ctx"], out)
         res["o_ctx"] = out
     if "phase2" in phases:
         T = wl.T

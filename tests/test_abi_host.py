@@ -32,6 +32,9 @@ def _shape(**kw):
     (dict(b=32704, L=32704 * 4), star.STAR_ERR_UNSUPPORTED_SHAPE),  # b not a multiple of 128
     (dict(B=0), star.STAR_ERR_INVALID_ARG),
     (dict(rope_theta=-1.0), star.STAR_ERR_INVALID_ARG),
+    (dict(anchor=-128), star.STAR_ERR_INVALID_ARG),              # negative anchor size
+    (dict(anchor=1000), star.STAR_ERR_UNSUPPORTED_SHAPE),         # anchor not a multiple of 128
+    (dict(anchor=32768 + 128), star.STAR_ERR_UNSUPPORTED_SHAPE),  # anchor larger than the block
 ])
 def test_shape_validation(kw, code):
     with pytest.raises(star.StarError) as e:
@@ -60,6 +63,16 @@ def test_workspace_sizes_for_every_workload():
         assert ws2 % 256 == 0 and wsd % 256 == 0 and wsd > 0
         with pytest.raises(star.StarError):
             star.star_workspace_size(sh, star.STAR_OP_PHASE2, wl.T_max + 1)
+
+
+def test_anchor_workspace_size():
+    """The anchor's keys roped at caller ids: bf16 [B][n-1][Hkv][a][d]; a = b when the shape says 0."""
+    for a in (0, 8192, 32768):
+        sh = _shape(B=2, anchor=a)
+        aa = a or 32768
+        assert star.star_workspace_size(sh, star.STAR_OP_PHASE1_ANCHOR) == 2 * 3 * 8 * aa * 128 * 2
+    one_block = _shape(L=32768, b=32768)
+    assert star.star_workspace_size(one_block, star.STAR_OP_PHASE1_ANCHOR) == 0
 
 
 def test_null_arguments_rejected_before_any_launch():
