@@ -44,7 +44,10 @@ Parity status per function (the pins live in ``tests/test_oracle_pins.py``):
   relative-shift invariance, identity at position 0, closed-form angles.
 * ``augmented_context``/``block_map`` pinned: hand-enumerated L=8, b=2 fixture; the
   anchor variants (anchor size a < b, per-block anchor position ids) by the
-  hand-enumerated L=12, b=4, a=2 fixture.
+  hand-enumerated L=12, b=4, a=2 fixture; a ragged last block by the L=10, b=4 fixture.
+* ragged / variable-length batches pinned: Phase-1 rows of a shorter context equal
+  the same rows of a longer one (causality); a batch equals its sequences run
+  alone; partials of missing blocks are empty and the merge equals brute force.
 * ``causal_attention``       pinned: torch scaled_dot_product_attention (causal, fp64).
 * ``phase1``/``phase1_rows`` pinned: n=1 equals textbook causal attention; n>1
   equals an independent full-length attention with the Star mask (library SDPA);
@@ -145,29 +148,32 @@ def augmented_context(L: int, b: int, pos_ctx=None, anchor: int | None = None, a
     ``anchor_pos`` [n-1, a] gives the anchor's position ids in block i >= 1
     (0-based), default the caller's ids of tokens 0..a-1.
 
+    A context that is not a multiple of b ends in a ragged block: the last of
+    the n = ceil(L / b) blocks holds the remaining L - (n-1) b tokens ([SA1] "问题
+    定义与记号" splits the context into blocks of b tokens; the ragged tail is the
+    plainest reading of a length that does not divide).
+
     Returns one dict per block (0-based ``i``) with ``tokens`` (context token
     index of every augmented row), ``pos`` (its position id) and ``kept`` (the
     augmented rows whose output and KV survive).
     """
-    if L % b:
-        raise ValueError("context length must be a multiple of the block size")
     a = b if anchor is None else int(anchor)
     if not 0 < a <= b:
         raise ValueError("anchor size must be in (0, b]")
-    n = L // b
+    n = -(-L // b)
     pos_ctx = np.arange(L, dtype=np.int64) if pos_ctx is None else np.asarray(pos_ctx, dtype=np.int64)
     if anchor_pos is not None:
         anchor_pos = np.asarray(anchor_pos, dtype=np.int64).reshape(n - 1, a)
     out = []
     for i in range(n):
-        own = np.arange(i * b, (i + 1) * b, dtype=np.int64)
+        own = np.arange(i * b, min((i + 1) * b, L), dtype=np.int64)
         if i == 0:
             tokens, pos = own, pos_ctx[own]
         else:
             tokens = np.concatenate([np.arange(a, dtype=np.int64), own])
             apos = pos_ctx[:a] if anchor_pos is None else anchor_pos[i - 1]
             pos = np.concatenate([apos, pos_ctx[own]])
-        out.append({"i": i, "tokens": tokens, "pos": pos, "kept": np.arange(len(tokens) - b, len(tokens))})
+        out.append({"i": i, "tokens": tokens, "pos": pos, "kept": np.arange(len(tokens) - len(own), len(tokens))})
     return out
 
 
@@ -262,7 +268,7 @@ def phase1_rows(rows, q_rows: np.ndarray, k: np.ndarray, v: np.ndarray, pos_ctx,
     """
     rows = np.asarray(rows, dtype=np.int64)
     L = k.shape[0]
-    n = L // b
+    n = -(-L // b)
     a = b if anchor is None else int(anchor)
     pos_ctx = np.arange(L, dtype=np.int64) if pos_ctx is None else np.asarray(pos_ctx, dtype=np.int64)
     if anchor_pos is not None:
@@ -272,13 +278,13 @@ def phase1_rows(rows, q_rows: np.ndarray, k: np.ndarray, v: np.ndarray, pos_ctx,
 
     def roped_block(i):
         if i not in cache:
-            tok = np.arange(i * b, (i + 1) * b)
+            tok = np.arange(i * b, min((i + 1) * b, L))
             cache[i] = rope_bf16(k[tok], pos_ctx[tok], theta)
         return cache[i]
 
     for i in np.unique(rows // b):
         sel = np.nonzero(rows // b == i)[0]
-        own = np.arange(i * b, (i + 1) * b)
+        own = np.arange(i * b, min((i + 1) * b, L))
         keys, vals, key_idx = roped_block(i), np.asarray(v[own], dtype=np.float64), own
         if i > 0:
             apos = pos_ctx[:a] if anchor_pos is None else anchor_pos[i - 1]
@@ -303,19 +309,24 @@ def append_tail(ck: np.ndarray, cv: np.ndarray, k_new: np.ndarray, v_new: np.nda
             np.concatenate([cv, np.asarray(v_new, dtype=np.float64)]))
 
 
-def phase2_partials(q_query: np.ndarray, pos_query, ck: np.ndarray, cv: np.ndarray, L: int, b: int, theta: float):
+def phase2_partials(q_query: np.ndarray, pos_query, ck: np.ndarray, cv: np.ndarray, L: int, b: int, theta: float,
+                    n_parts: int | None = None):
     """Per-block local attention of the query rows ([SA1] "Phase 2: 局部注意力与本地统计量").
 
     ck/cv: the cache [L + T, Hkv, d] with the query tokens' K/V already appended
     (tail of the last block).  Query token t (cache index L + t) sees every key of
-    blocks 1..n-1 and, in the last block, its b context keys plus tail keys L..L+t.
-    Returns O_part [n, T, Hq, d] and LSE_part [n, T, Hq].
+    blocks 1..n-1 and, in the last block, its context keys plus tail keys L..L+t.
+    n = ceil(L / b); with ``n_parts`` > n (a batch whose longest sequence has more
+    blocks) the partials of the missing blocks are empty: O = 0, LSE = -inf, which
+    the merge skips ([SA1] "数值稳定性").
+    Returns O_part [n_parts, T, Hq, d] and LSE_part [n_parts, T, Hq].
     """
     T = q_query.shape[0]
-    n = L // b
+    n = -(-L // b)
+    n_parts = n if n_parts is None else int(n_parts)
     qr = rope_bf16(q_query, pos_query, theta)
-    O_part = np.zeros((n, T) + q_query.shape[1:])
-    LSE_part = np.zeros((n, T, q_query.shape[1]))
+    O_part = np.zeros((n_parts, T) + q_query.shape[1:])
+    LSE_part = np.full((n_parts, T, q_query.shape[1]), -np.inf)
     row_idx = L + np.arange(T)
     for i in range(n):
         lo, hi = i * b, (i + 1) * b if i < n - 1 else ck.shape[0]
@@ -385,25 +396,32 @@ def run_star(inp: dict, L: int, b: int, theta: float, with_phase1: bool = True, 
     [B, T, Hq, d], k_query/v_query [B, T, Hkv, d], pos_query [B, T], q_dec
     [S, B, 1, Hq, d], k_dec/v_dec [S, B, 1, Hkv, d], pos_dec [S, B]; optionally
     anchor_pos [B, n-1, a] (the anchor's position ids per block, see
-    ``augmented_context``).  ``anchor``: the anchor size a (default b).
+    ``augmented_context``) and seq_len [B] (each sequence's context length; the
+    context arrays are then padded to L and the rows past a sequence's length are
+    ignored, its outputs there are 0).  ``anchor``: the anchor size a (default b).
+    Every sequence has ceil(L / b) partials; those past its own blocks are empty.
     """
     B = inp["q_ctx"].shape[0]
     res: dict[str, list] = {k: [] for k in ("o_ctx", "cache_k", "cache_v", "o_part", "lse_part",
                                             "o_query", "lse_query", "o_dec", "lse_dec")}
+    n_parts = -(-L // b)
     for bi in range(B):
+        Ls = int(inp["seq_len"][bi]) if inp.get("seq_len") is not None else L
         if with_phase1:
             apos = inp["anchor_pos"][bi] if inp.get("anchor_pos") is not None else None
-            O1, ck, cv = phase1(inp["q_ctx"][bi], inp["k_ctx"][bi], inp["v_ctx"][bi], inp["pos_ctx"][bi], b, theta,
-                                anchor, apos)
-            res["o_ctx"].append(O1)
+            O1, ck, cv = phase1(inp["q_ctx"][bi][:Ls], inp["k_ctx"][bi][:Ls], inp["v_ctx"][bi][:Ls],
+                                inp["pos_ctx"][bi][:Ls], b, theta, anchor, apos)
+            Opad = np.zeros(inp["q_ctx"][bi].shape)
+            Opad[:Ls] = O1
+            res["o_ctx"].append(Opad)
         else:
-            tok = np.arange(L)
-            ck = rope_bf16(inp["k_ctx"][bi], inp["pos_ctx"][bi][tok], theta)
-            cv = np.asarray(inp["v_ctx"][bi], dtype=np.float64)
+            tok = np.arange(Ls)
+            ck = rope_bf16(inp["k_ctx"][bi][:Ls], inp["pos_ctx"][bi][tok], theta)
+            cv = np.asarray(inp["v_ctx"][bi][:Ls], dtype=np.float64)
         res["cache_k"].append(ck)
         res["cache_v"].append(cv)
         ck, cv = append_tail(ck, cv, inp["k_query"][bi], inp["v_query"][bi], inp["pos_query"][bi], theta)
-        Op, Lp = phase2_partials(inp["q_query"][bi], inp["pos_query"][bi], ck, cv, L, b, theta)
+        Op, Lp = phase2_partials(inp["q_query"][bi], inp["pos_query"][bi], ck, cv, Ls, b, theta, n_parts)
         Oq, Lq = lse_merge(Op, Lp)
         res["o_part"].append(Op)
         res["lse_part"].append(Lp)
@@ -425,6 +443,8 @@ def run_star(inp: dict, L: int, b: int, theta: float, with_phase1: bool = True, 
             out[k] = np.stack(vals, axis=1)          # [n, B, ...]
         elif k in ("o_dec", "lse_dec"):
             out[k] = np.stack(vals, axis=1)          # [S, B, ...]
+        elif k in ("cache_k", "cache_v") and len({v.shape for v in vals}) > 1:
+            out[k] = vals                            # per-sequence lengths differ
         else:
             out[k] = np.stack(vals)
     return out

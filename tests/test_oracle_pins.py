@@ -547,3 +547,108 @@ def test_planted_anchor_mistake_is_caught(monkeypatch):
             assert diff < 1e-12
         else:
             assert diff > 1e-2, (name, diff)
+
+
+# ---------------------------------------------------------------------------
+# Ragged last block, variable-length batches
+# ---------------------------------------------------------------------------
+
+def test_ragged_block_matches_hand_fixture():
+    g = _golden("ragged_L10_b4.json")
+    blocks = oracle.augmented_context(g["L"], g["b"])
+    assert len(blocks) == g["n"]
+    assert [blk["tokens"].tolist() for blk in blocks] == g["augmented_tokens"]
+    assert [blk["pos"].tolist() for blk in blocks] == g["augmented_pos"]
+    assert [blk["kept"].tolist() for blk in blocks] == g["kept"]
+    kept = np.concatenate([blk["tokens"][blk["kept"]] for blk in blocks])
+    assert kept.tolist() == g["cached_tokens"]
+
+
+def _seq(seed, L, Hq=4, Hkv=2, d=16):
+    rng = np.random.default_rng(seed)
+    return _bf16_values(rng, (L, Hq, d)), _bf16_values(rng, (L, Hkv, d)), _bf16_values(rng, (L, Hkv, d))
+
+
+def test_phase1_of_a_shorter_context_is_the_prefix_of_a_longer_one():
+    """Row t's output depends only on the anchor and its own block up to t, so cutting
+    the context at any length (a ragged last block) keeps the kept rows' outputs."""
+    theta, b = 500000.0, 16
+    q, k, v = _seq(31, 64)
+    pos = np.arange(64)
+    O_full, ck_full, _ = oracle.phase1(q, k, v, pos, b, theta)
+    for Ls in (17, 40, 47, 63):
+        O, ck, cv = oracle.phase1(q[:Ls], k[:Ls], v[:Ls], pos[:Ls], b, theta)
+        np.testing.assert_allclose(O, O_full[:Ls], rtol=0, atol=1e-12, err_msg=str(Ls))
+        assert np.array_equal(ck, ck_full[:Ls])
+        rows = np.array([0, Ls // 2, Ls - 1])
+        np.testing.assert_allclose(oracle.phase1_rows(rows, q[rows], k[:Ls], v[:Ls], pos[:Ls], b, theta), O[rows],
+                                   rtol=0, atol=1e-12)
+
+
+def test_ragged_phase2_merge_equals_brute_force_with_empty_partials():
+    theta, b, T = 500000.0, 16, 5
+    q, k, v = _seq(32, 40)
+    qq, kq, vq = _seq(33, T)
+    pos, qpos = np.arange(40), 40 + np.arange(T)
+    _, ck, cv = oracle.phase1(q, k, v, pos, b, theta)
+    ck, cv = oracle.append_tail(ck, cv, kq, vq, qpos, theta)
+    Op, Lp = oracle.phase2_partials(qq, qpos, ck, cv, 40, b, theta, n_parts=5)
+    assert Op.shape[0] == 5 and np.all(Lp[3:] == -np.inf) and np.all(Op[3:] == 0)
+    O, LSE = oracle.lse_merge(Op, Lp)
+    qr = oracle.round_to_bf16(rope_complex(qq, qpos, theta))
+    mask = np.arange(ck.shape[0])[None, :] <= (40 + np.arange(T))[:, None]
+    np.testing.assert_allclose(O, sdpa(qr, ck, cv, mask), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(LSE, lse_lib(qr, ck, mask), rtol=0, atol=1e-12)
+
+
+def _varlen_batch(lens, L, b, T, S, seed=34):
+    rng = np.random.default_rng(seed)
+    B = len(lens)
+    f = lambda *sh: _bf16_values(rng, sh)
+    inp = {"q_ctx": f(B, L, 4, 16), "k_ctx": f(B, L, 2, 16), "v_ctx": f(B, L, 2, 16),
+           "pos_ctx": np.tile(np.arange(L), (B, 1)), "seq_len": np.array(lens),
+           "q_query": f(B, T, 4, 16), "k_query": f(B, T, 2, 16), "v_query": f(B, T, 2, 16),
+           "pos_query": np.stack([Ls + np.arange(T) for Ls in lens]),
+           "q_dec": f(S, B, 1, 4, 16), "k_dec": f(S, B, 1, 2, 16), "v_dec": f(S, B, 1, 2, 16),
+           "pos_dec": np.stack([[Ls + T + s for Ls in lens] for s in range(S)])}
+    return inp
+
+
+def test_varlen_batch_equals_each_sequence_alone():
+    theta, L, b, T, S = 500000.0, 64, 16, 3, 2
+    lens = [64, 33, 16, 50]
+    inp = _varlen_batch(lens, L, b, T, S)
+    ref = oracle.run_star(inp, L, b, theta)
+    for bi, Ls in enumerate(lens):
+        one = {k: (v[bi:bi + 1] if k not in ("q_dec", "k_dec", "v_dec", "pos_dec") else v[:, bi:bi + 1])
+               for k, v in inp.items() if k != "seq_len"}
+        one = {k: (v[:, :Ls] if k in ("q_ctx", "k_ctx", "v_ctx", "pos_ctx") else v) for k, v in one.items()}
+        alone = oracle.run_star(one, Ls, b, theta)
+        np.testing.assert_array_equal(ref["o_ctx"][bi][:Ls], alone["o_ctx"][0])
+        assert np.all(ref["o_ctx"][bi][Ls:] == 0)
+        n = -(-Ls // b)
+        np.testing.assert_array_equal(ref["o_part"][:n, bi], alone["o_part"][:, 0])
+        assert np.all(ref["lse_part"][n:, bi] == -np.inf)
+        for key in ("o_query", "lse_query"):
+            np.testing.assert_allclose(ref[key][bi], alone[key][0], rtol=0, atol=1e-12)
+        for key in ("o_dec", "lse_dec"):
+            np.testing.assert_allclose(ref[key][:, bi], alone[key][:, 0], rtol=0, atol=1e-12)
+
+
+def test_planted_tail_at_the_padded_end_is_caught(monkeypatch):
+    """Placing a short sequence's query tail after the padded capacity instead of its own
+    context end leaves a gap of keys it may not see; the brute-force pin catches it."""
+    theta, b, T = 500000.0, 16, 4
+    q, k, v = _seq(35, 40)
+    qq, kq, vq = _seq(36, T)
+    pos, qpos = np.arange(40), 40 + np.arange(T)
+    _, ck, cv = oracle.phase1(q, k, v, pos, b, theta)
+    ck, cv = oracle.append_tail(ck, cv, kq, vq, qpos, theta)
+    qr = oracle.round_to_bf16(rope_complex(qq, qpos, theta))
+    mask = np.arange(ck.shape[0])[None, :] <= (40 + np.arange(T))[:, None]
+    want = sdpa(qr, ck, cv, mask)
+    # wrong: the tail believed to start at 48 (the capacity 3 * b) -> rows see 8 extra keys
+    Op, Lp = oracle.phase2_partials(qq, qpos, ck, cv, 48, b, theta)
+    O, _ = oracle.lse_merge(Op, Lp)
+    assert np.abs(O - want).max() > 1e-2
+
