@@ -49,12 +49,23 @@ class StarShape(ctypes.Structure):
         ("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("d", ctypes.c_int32),
         ("L", ctypes.c_int32), ("b", ctypes.c_int32), ("n", ctypes.c_int32), ("T_max", ctypes.c_int32),
         ("page_tokens", ctypes.c_int32), ("rope_theta", ctypes.c_double), ("anchor", ctypes.c_int32),
+        ("seq_len", ctypes.POINTER(ctypes.c_int32)),
     ]
 
     @classmethod
-    def make(cls, B, Hq, Hkv, d, L, b, T_max, page_tokens=256, rope_theta=500000.0, anchor=0) -> "StarShape":
-        """anchor: the anchor size a (the first a tokens of block 1); 0 means b."""
-        return cls(B, Hq, Hkv, d, L, b, L // b if b else 0, T_max, page_tokens, rope_theta, anchor)
+    def make(cls, B, Hq, Hkv, d, L, b, T_max, page_tokens=256, rope_theta=500000.0, anchor=0,
+             seq_len=None) -> "StarShape":
+        """anchor: the anchor size a (the first a tokens of block 1); 0 means b.
+        seq_len: per-sequence context lengths (B ints, each in [1, L]) or None; L is then the
+        capacity and each sequence's tail starts at its own length."""
+        sh = cls(B, Hq, Hkv, d, L, b, L // b if b else 0, T_max, page_tokens, rope_theta, anchor)
+        if seq_len is not None:
+            lens = [int(x) for x in seq_len]
+            if len(lens) != B:
+                raise ValueError(f"seq_len has {len(lens)} entries for B = {B}")
+            sh._seq_len_buf = (ctypes.c_int32 * B)(*lens)   # kept alive with the shape
+            sh.seq_len = ctypes.cast(sh._seq_len_buf, ctypes.POINTER(ctypes.c_int32))
+        return sh
 
 
 class StarCache(ctypes.Structure):

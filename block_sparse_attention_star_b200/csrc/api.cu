@@ -68,6 +68,14 @@ int check_shape(const star_shape* s) {
   if (s->page_tokens % 128) return fail(STAR_ERR_UNSUPPORTED_SHAPE, "page_tokens (%d) must be a multiple of 128", s->page_tokens);
   if (s->b % s->page_tokens)
     return fail(STAR_ERR_UNSUPPORTED_SHAPE, "b (%d) must be a multiple of page_tokens (%d)", s->b, s->page_tokens);
+  if (s->seq_len) {
+    if (s->B > star::kMaxVarB)
+      return fail(STAR_ERR_UNSUPPORTED_SHAPE, "per-sequence lengths are supported for B <= %d (B = %d)", star::kMaxVarB,
+                  s->B);
+    for (int i = 0; i < s->B; ++i)
+      if (s->seq_len[i] < 1 || s->seq_len[i] > s->L)
+        return fail(STAR_ERR_INVALID_ARG, "seq_len[%d] = %d outside [1, L = %d]", i, s->seq_len[i], s->L);
+  }
   if (s->anchor < 0) return fail(STAR_ERR_INVALID_ARG, "anchor size (%d) must not be negative", s->anchor);
   if (s->anchor > s->b || s->anchor % 128)
     return fail(STAR_ERR_UNSUPPORTED_SHAPE, "anchor size (%d) must be a multiple of 128 and at most b (%d)", s->anchor,
@@ -155,6 +163,16 @@ size_t phase2_ws_bytes(const star_shape* s, int T) {
 }
 
 int anchor_of(const star_shape* s) { return s->anchor ? s->anchor : s->b; }
+
+// Per-sequence context lengths as shifts of the capacity frame (delta = L_s - L).
+star::SeqShift shift_of(const star_shape* s) {
+  star::SeqShift sh;
+  memset(&sh, 0, sizeof(sh));
+  sh.on = s->seq_len ? 1 : 0;
+  if (sh.on)
+    for (int i = 0; i < s->B; ++i) sh.delta[i] = s->seq_len[i] - s->L;
+  return sh;
+}
 
 // The anchor's keys, roped at caller-given ids, per (sequence, block 2..n): bf16 [B][n-1][Hkv][a][d].
 size_t anchor_ws_bytes(const star_shape* s) {
@@ -245,8 +263,12 @@ int star_kv_append(const star_shape* shape, const star_cache* cache, const void*
   if (start < 0 || ntok < 0) return fail(STAR_ERR_INVALID_ARG, "start and ntok must be >= 0");
   if ((int64_t)start + ntok > (int64_t)shape->L + shape->T_max)
     return fail(STAR_ERR_CAPACITY, "slots [%d, %d) exceed L + T_max = %d", start, start + ntok, shape->L + shape->T_max);
+  if (shape->seq_len && start < shape->L)
+    return fail(STAR_ERR_INVALID_ARG, "with per-sequence lengths, start (%d) counts from the capacity L = %d and "
+                "must be >= L", start, shape->L);
+  const star::SeqShift sh = shift_of(shape);
   cudaError_t e = star::launch_rope_append(k, v, pos, shape->B, ntok, start, shape->Hkv, shape->d, view(shape, cache),
-                                           rope_table(shape), (cudaStream_t)stream);
+                                           rope_table(shape), (cudaStream_t)stream, &sh);
   return e == cudaSuccess ? STAR_OK : cuda_fail(e, "kv_append launch");
 }
 
@@ -278,8 +300,9 @@ int star_phase1_encode_anchored(const star_shape* shape, const star_cache* cache
   const star::RopeTable rt = rope_table(shape);
   cudaError_t e = star::launch_rope_append(k, v, pos_ctx, shape->B, shape->L, 0, shape->Hkv, shape->d, cv, rt, st);
   if (e != cudaSuccess) return cuda_fail(e, "phase1 kv append");
+  const star::SeqShift sh = shift_of(shape);
   e = star::launch_zero_slots(shape->B, shape->L, shape->L + (int)round_up(shape->T_max, 128), shape->Hkv, shape->d,
-                              cv, st);
+                              cv, st, &sh);
   if (e != cudaSuccess) return cuda_fail(e, "phase1 tail clear");
   const int anchor = anchor_of(shape);
   const bool own_anchor_ids = anchor_pos && shape->n > 1;
@@ -292,6 +315,7 @@ int star_phase1_encode_anchored(const star_shape* shape, const star_cache* cache
   a.mode = 0;
   a.anchor = anchor;
   a.anchor_k = own_anchor_ids ? ws : nullptr;
+  a.shift = sh;
   a.B = shape->B;
   a.Hq = shape->Hq;
   a.Hkv = shape->Hkv;
@@ -339,7 +363,8 @@ int star_phase2_partial(const star_shape* shape, const star_cache* cache, const 
   if (k) {
     STAR_REQUIRE_PTR(k, "k");
     STAR_REQUIRE_PTR(v, "v");
-    cudaError_t e = star::launch_rope_append(k, v, q_pos, shape->B, T, shape->L, shape->Hkv, shape->d, cv, rt, st);
+    const star::SeqShift shq = shift_of(shape);
+    cudaError_t e = star::launch_rope_append(k, v, q_pos, shape->B, T, shape->L, shape->Hkv, shape->d, cv, rt, st, &shq);
     if (e != cudaSuccess) return cuda_fail(e, "phase2 kv append");
   }
   const int cpb = phase2_chunks_per_block(shape, T);
@@ -354,6 +379,7 @@ int star_phase2_partial(const star_shape* shape, const star_cache* cache, const 
   star::AttnLaunch a;
   memset(&a, 0, sizeof(a));
   a.mode = 1;
+  a.shift = shift_of(shape);
   a.B = shape->B;
   a.Hq = shape->Hq;
   a.Hkv = shape->Hkv;
@@ -409,6 +435,9 @@ int star_decode_step(const star_shape* shape, const star_cache* cache, const voi
   if (lse_out && (reinterpret_cast<uintptr_t>(lse_out) & 3u)) return fail(STAR_ERR_ALIGNMENT, "lse_out is not 4-byte aligned");
   if (cur_len < 0 || cur_len >= shape->L + shape->T_max)
     return fail(STAR_ERR_CAPACITY, "cur_len %d outside [0, L + T_max = %d)", cur_len, shape->L + shape->T_max);
+  if (shape->seq_len && cur_len < shape->L)
+    return fail(STAR_ERR_INVALID_ARG, "with per-sequence lengths, cur_len (%d) counts from the capacity L = %d and "
+                "must be >= L", cur_len, shape->L);
   const size_t need = decode_ws_bytes(shape);
   if (ws_bytes < need) return fail(STAR_ERR_CAPACITY, "workspace %zu bytes < %zu needed", ws_bytes, need);
   cudaStream_t st = (cudaStream_t)stream;
@@ -430,6 +459,7 @@ int star_decode_step(const star_shape* shape, const star_cache* cache, const voi
   a.v_new = v;
   a.pos = pos;
   a.n_keys = n_keys;
+  a.shift = shift_of(shape);
   a.chunk = chunk;
   a.cache = cv;
   a.o_ws = reinterpret_cast<float*>(ws);

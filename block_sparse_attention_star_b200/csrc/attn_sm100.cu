@@ -74,6 +74,7 @@ struct Params {
   int num_items;
   // Phase-1 anchor: its size, and whether its keys come from the tmKA map (roped at caller ids)
   int anchor, anchor_k_on;
+  SeqShift sh;  // per-sequence context lengths L + delta[bi] (sh.on = 0: every sequence has L)
   float scale_log2;
   double inv_freq[kMaxHalfDim];
 };
@@ -81,7 +82,9 @@ struct Params {
 struct Item {
   int bi, g;
   int a_start, a_tiles;   // first run of key tiles (cache index of its first key, tile count)
-  int b_start, b_tiles;   // second run
+  int a_end;              // keys of the first run at or past a_end are not visible
+  int b_start, b_tiles;   // second run (tiles start at b_start rounded down to 128)
+  int skip;               // mode 0: the item's rows are all past the sequence's context
   int part;               // Phase 2: output part (global chunk index)
   int r0;                 // Phase 1: context index of the tile's first row
   int hp;                 // Phase 1: head pair in the group; Phase 2: row-tile pair
@@ -90,9 +93,12 @@ struct Item {
 // Work items.  Phase 1, per (sequence, KV head): items of blocks 2..n first,
 // then block 1's, each run ordered by descending q-tile, so item cost falls
 // monotonically and the round-robin assignment to CTAs stays balanced.
+__device__ __forceinline__ int ctx_len(const Params& p, int bi) { return p.L + (p.sh.on ? p.sh.delta[bi] : 0); }
+
 template <int MODE>
 __device__ __forceinline__ Item decode_item(const Params& p, int idx) {
   Item it;
+  it.skip = 0;
   if (MODE == 0) {
     const int nqt = p.b / kRows;
     const int npairs = p.G / 2;
@@ -117,10 +123,12 @@ __device__ __forceinline__ Item decode_item(const Params& p, int idx) {
     }
     it.a_start = 0;
     it.a_tiles = (i > 0) ? p.anchor / kRows : 0;  // the anchor: the first a keys of block 1
+    it.a_end = p.anchor;
     it.b_start = i * p.b;
     it.b_tiles = t + 1;
     it.part = i;
     it.r0 = i * p.b + t * kRows;
+    it.skip = it.r0 >= ctx_len(p, it.bi);  // a shorter sequence: every row of the tile is padding
   } else {
     it.hp = idx % p.npairs;
     int rest = idx / p.npairs;
@@ -128,19 +136,23 @@ __device__ __forceinline__ Item decode_item(const Params& p, int idx) {
     rest /= p.Hkv;
     it.bi = rest % p.B;
     const int c = rest / p.B;
+    const int Ls = ctx_len(p, it.bi);
     it.part = c;
+    // The chunk's context keys, cut at the sequence's length; the tail (query tokens,
+    // cache indices Ls ..) follows the chunk that holds the last context key.
     it.a_start = c * p.chunk_keys;
-    it.a_tiles = p.chunk_keys / kKeys;
-    const bool last = (c == p.n * p.chunks_per_block - 1);
-    it.b_start = p.L;
-    it.b_tiles = last ? p.tail_tiles : 0;
+    it.a_end = min(it.a_start + p.chunk_keys, Ls);
+    it.a_tiles = it.a_end > it.a_start ? (it.a_end - it.a_start + kKeys - 1) / kKeys : 0;
+    const bool last = (c == (Ls - 1) / p.chunk_keys);
+    it.b_start = Ls;
+    it.b_tiles = last ? (Ls % kKeys + p.Ntok + kKeys - 1) / kKeys : 0;
     it.r0 = 0;
   }
   return it;
 }
 
 __device__ __forceinline__ int tile_key0(const Item& it, int j) {
-  return j < it.a_tiles ? it.a_start + j * kKeys : it.b_start + (j - it.a_tiles) * kKeys;
+  return j < it.a_tiles ? it.a_start + j * kKeys : (it.b_start & ~(kKeys - 1)) + (j - it.a_tiles) * kKeys;
 }
 
 struct RowInfo {
@@ -167,7 +179,7 @@ __device__ __forceinline__ RowInfo row_info(const Params& p, const Item& it, int
     r.valid = (rt < p.NTT * p.NHT) && (hl < p.G) && (t < p.Ntok);
     r.head = it.g * p.G + (r.valid ? hl : 0);
     r.tok = r.valid ? t : 0;
-    r.cache_idx = r.valid ? p.L + t : INT_MAX;
+    r.cache_idx = r.valid ? ctx_len(p, it.bi) + t : INT_MAX;
   }
   r.pos = r.valid ? p.q_pos[(size_t)it.bi * p.Ntok + r.tok] : 0;
   if (!r.valid) r.cache_idx = INT_MAX;
@@ -289,6 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int idx = blockIdx.x; idx < p.num_items && ok; idx += gridDim.x) {
         const Item it = decode_item<MODE>(p, idx);
+        if (it.skip) continue;
         const int nt = it.a_tiles + it.b_tiles;
         for (int j = 0; j < nt && ok; ++j) {
           const int k0 = tile_key0(it, j);
@@ -344,8 +357,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t qc = 0;
       bool ok = true;
-      for (int idx = blockIdx.x; idx < p.num_items && ok; idx += gridDim.x, ++qc) {
+      for (int idx = blockIdx.x; idx < p.num_items && ok; idx += gridDim.x) {
         const Item it = decode_item<MODE>(p, idx);
+        if (it.skip) continue;
         if (qc > 0) ok = mbar_wait(q_empty, (qc - 1) & 1, kDevTimeoutProducer);
         if (!ok) break;
 #pragma unroll
@@ -356,6 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_4d(smem + S::kQ0 + w * S::kTile + h * (kRows * 128), &tmQ, &q_full[w], h * 64,
                         it.g * p.G + 2 * it.hp + w, it.r0, it.bi);
         }
+        ++qc;
       }
       // Drain: the last loads have landed before the CTA exits.
       if (qc > 0) {
@@ -413,6 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int idx = blockIdx.x; idx < p.num_items && ok; idx += gridDim.x) {
         const Item it = decode_item<MODE>(p, idx);
         const int nt = it.a_tiles + it.b_tiles;
+        if (it.skip || nt == 0) continue;  // padding rows, or a Phase-2 chunk past the sequence
         ok = mbar_wait(&q_full[0], qph, kDevTimeoutMma) && mbar_wait(&q_full[1], qph, kDevTimeoutMma);
         if (!ok) break;
         qph ^= 1;
@@ -477,14 +493,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
 
     for (int idx = blockIdx.x; idx < p.num_items && ok; idx += gridDim.x) {
-      int nt, a_tiles, a_start, b_start, cache_idx;
+      int nt, a_tiles, a_start, a_end, b_start, cache_idx;
       {
         const Item it = decode_item<MODE>(p, idx);
+        if (it.skip) continue;
         const RowInfo ri = row_info<MODE>(p, it, wg, row);
-        if (MODE == 1) load_q_row<D>(p, it, ri, sQ, row);  // mode 0: Q arrives by TMA
         nt = it.a_tiles + it.b_tiles;
+        if (MODE == 1 && nt == 0) {
+          // A chunk past the sequence's context: an empty partial (O = 0, LSE = -inf),
+          // which the merge skips.
+          if (ri.valid) {
+            const size_t rowoff = (((size_t)it.part * p.B + it.bi) * p.Ntok + ri.tok) * p.Hq + ri.head;
+            float4* d4 = reinterpret_cast<float4*>(p.out_f32 + rowoff * D);
+#pragma unroll
+            for (int e = 0; e < D / 4; ++e) d4[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+            p.lse_f32[rowoff] = -INFINITY;
+          }
+          continue;
+        }
+        if (MODE == 1) load_q_row<D>(p, it, ri, sQ, row);  // mode 0: Q arrives by TMA
         a_tiles = it.a_tiles;
         a_start = it.a_start;
+        a_end = it.a_end;
         b_start = it.b_start;
         cache_idx = ri.cache_idx;
       }
@@ -504,12 +534,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
         tmem_ld_wait();
-        const int k0 = j < a_tiles ? a_start + j * kKeys : b_start + (j - a_tiles) * kKeys;
-        if (k0 + kKeys - 1 > cache_idx) {
-          const int lim = cache_idx - k0;  // keys k0 + c with c > lim are not visible
+        // Visible keys of this tile: lo <= key <= hi (the run's range, and causal by
+        // cache index).  The second run's tiles start at b_start rounded down to 128.
+        int k0, lo, hi;
+        if (j < a_tiles) {
+          k0 = a_start + j * kKeys;
+          lo = a_start;
+          hi = min(a_end - 1, cache_idx);
+        } else {
+          k0 = (b_start & ~(kKeys - 1)) + (j - a_tiles) * kKeys;
+          lo = b_start;
+          hi = cache_idx;
+        }
+        if (k0 < lo || k0 + kKeys - 1 > hi) {
+          const int clo = lo - k0, chi = hi - k0;  // keys k0 + c with c outside [clo, chi] are not visible
 #pragma unroll
           for (int c = 0; c < kKeys; ++c)
-            if (c > lim) sr[c] = __float_as_uint(-INFINITY);
+            if (c < clo || c > chi) sr[c] = __float_as_uint(-INFINITY);
         }
         // Row max of the raw scores (scale > 0 commutes with max); 4 independent chains.
         float mx[4];
@@ -592,6 +633,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv_l = (lr > 0.f) ? 1.f / lr : 0.f;
       if (MODE == 0) {
         bf16* dst = p.out_bf16 + (((size_t)it.bi * p.L + ri.tok) * p.Hq + ri.head) * D;
+        const bool keep = ri.tok < ctx_len(p, it.bi);  // rows past a shorter sequence are padding
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
@@ -602,8 +644,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 16; ++e)
             w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
           uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+          if (keep) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) d4[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+            for (int e = 0; e < 4; ++e) d4[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+          }
         }
         // O_w is read: the next item's first P V may overwrite it.
         tc_fence_before();
@@ -784,6 +828,7 @@ cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t st, const char** 
   }
   CUtensorMap mka = mk;  // unused unless the anchor's keys are roped at caller ids
   p.anchor = a.mode == 0 ? a.anchor : 0;
+  p.sh = a.shift;
   p.anchor_k_on = (a.mode == 0 && a.anchor_k && a.n > 1) ? 1 : 0;
   if (p.anchor_k_on && !make_anchor_map(&mka, a.anchor_k, a.d, a.anchor, a.Hkv, a.B * (a.n - 1))) {
     if (why) *why = "cuTensorMapEncodeTiled failed for the anchor's keys";

@@ -66,6 +66,7 @@ struct DecParams {
   int B, Hq, Hkv, n_keys, chunk, nchunks;
   int item_base, num_items;  // this launch: items [item_base, num_items)
   float scale_log2;
+  SeqShift sh;               // sequence bi has n_keys + delta[bi] keys (sh.on = 0: all n_keys)
   double inv_freq[kMaxHalfDim];
 };
 
@@ -91,6 +92,8 @@ struct DecSmem {
 
 struct DecItem {
   int bi, g, c, k_begin, k_end, ntiles;
+  int n_keys;  // keys of this sequence
+  int last;    // the chunk holds the sequence's last key (the new token's slot)
 };
 
 __device__ __forceinline__ DecItem dec_item(const DecParams& p, int idx) {
@@ -98,9 +101,12 @@ __device__ __forceinline__ DecItem dec_item(const DecParams& p, int idx) {
   it.c = idx % p.nchunks;
   it.g = (idx / p.nchunks) % p.Hkv;
   it.bi = idx / (p.nchunks * p.Hkv);
+  it.n_keys = p.n_keys + (p.sh.on ? p.sh.delta[it.bi] : 0);
   it.k_begin = it.c * p.chunk;
-  it.k_end = min(it.k_begin + p.chunk, p.n_keys);
-  it.ntiles = (it.k_end - it.k_begin + kTileKeys - 1) / kTileKeys;
+  it.k_end = min(it.k_begin + p.chunk, it.n_keys);
+  // A chunk past a shorter sequence's keys is empty (0 tiles): its partial is O = 0, LSE = -inf.
+  it.ntiles = it.k_end > it.k_begin ? (it.k_end - it.k_begin + kTileKeys - 1) / kTileKeys : 0;
+  it.last = (it.c == (it.n_keys - 1) / p.chunk);
   return it;
 }
 
@@ -206,8 +212,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const DecItem it = dec_item(p, first + ii * gridDim.x);
     const int tpos = p.pos[it.bi];
     // Append the new token (head g) when this item holds the cache's last key.
-    if (it.c == p.nchunks - 1) {
-      const int slot_abs = p.n_keys - 1;
+    if (it.last) {
+      const int slot_abs = it.n_keys - 1;
       const int page = p.page_table[(size_t)it.bi * p.max_pages + slot_abs / p.P];
       if (page < 0 || page >= p.num_pages) {
         if (threadIdx.x == 0) record_error(kDevBadPage);
@@ -376,8 +382,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       return true;
     };
 
+    uint32_t nred = 0;  // items that took the row-sum barrier
     for (int ii = 0; ii < n_my && ok; ++ii) {
       const DecItem it = dec_item(p, first + ii * gridDim.x);
+      if (it.ntiles == 0) {
+        // A chunk past this sequence's keys: an empty partial (O = 0, LSE = -inf), which
+        // the merge skips; no tile of it is loaded or multiplied.
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const size_t row = (size_t)it.bi * p.Hq + it.g * G + h;
+          if (kt < D) p.o_ws[((size_t)it.c * rows + row) * D + kt] = 0.f;
+          if (kt == h) p.lse_ws[(size_t)it.c * rows + row] = -INFINITY;
+        }
+        continue;
+      }
       float m_run[G], lu[G], lr[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) {
@@ -457,7 +475,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(red_bar);
-      ok = __all_sync(0xffffffffu, mbar_wait(red_bar, ii & 1, kDevTimeoutSoftmax));
+      ok = __all_sync(0xffffffffu, mbar_wait(red_bar, nred & 1, kDevTimeoutSoftmax));
+      ++nred;
       if (!ok) break;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
@@ -598,6 +617,7 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t st) {
   p.item_base = 0;
   p.num_items = 0;
   p.scale_log2 = a.scale_log2;
+  p.sh = a.shift;
   for (int j = 0; j < kMaxHalfDim; ++j) p.inv_freq[j] = j < a.d / 2 ? a.rope.inv_freq[j] : 0.0;
   if (a.chunk <= 0 || a.chunk % kTileKeys != 0 || a.cache.P % kTileKeys != 0) return cudaErrorInvalidValue;
   CUtensorMap mk, mv;

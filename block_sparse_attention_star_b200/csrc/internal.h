@@ -8,6 +8,15 @@
 namespace star {
 
 constexpr int kMaxHalfDimHost = 64;
+constexpr int kMaxVarB = 256;   // sequences of a batch with per-sequence lengths (passed by value)
+
+// Per-sequence shift of cache indices: a batch with per-sequence context lengths
+// L_s keeps sequence s's tail at L_s, i.e. index x of the capacity frame maps to
+// x + delta[s] with delta[s] = L_s - L.  on = 0: every sequence has L tokens.
+struct SeqShift {
+  int on;
+  int delta[kMaxVarB];
+};
 
 struct RopeTable {
   double inv_freq[kMaxHalfDimHost];   // theta^(-2j/d), j < d/2
@@ -26,14 +35,18 @@ struct CacheView {
 // --- rope_append.cu -------------------------------------------------------
 // RoPE(K) at `pos` and copy of V for ntok tokens per sequence, written at cache
 // slots [start, start + ntok).  k/v: [B][ntok][Hkv][d] bf16, pos: [B][ntok].
+// shift (may be NULL): sequence s writes slots [start + delta[s], ...).
 cudaError_t launch_rope_append(const void* k, const void* v, const int32_t* pos, int B, int ntok, int start,
-                               int Hkv, int d, const CacheView& c, const RopeTable& rt, cudaStream_t st);
+                               int Hkv, int d, const CacheView& c, const RopeTable& rt, cudaStream_t st,
+                               const SeqShift* shift = nullptr);
 // RoPE of all H query heads of ntok tokens: out = rotate(q) at pos (out may be q).
 // q/out: [B][ntok][H][d] bf16, pos: [B][ntok].
 cudaError_t launch_rope_q(const void* q, const int32_t* pos, int B, int ntok, int H, int d, void* out,
                           const RopeTable& rt, cudaStream_t st);
 // Zero cache slots [from, to) of every sequence (K and V).
-cudaError_t launch_zero_slots(int B, int from, int to, int Hkv, int d, const CacheView& c, cudaStream_t st);
+// shift (may be NULL): sequence s clears slots [from + delta[s], to).
+cudaError_t launch_zero_slots(int B, int from, int to, int Hkv, int d, const CacheView& c, cudaStream_t st,
+                              const SeqShift* shift = nullptr);
 // c' position ids [B][L + (n-1) a] (anchor = the first a tokens) and block map [B][L][3].
 cudaError_t launch_build_positions(const int32_t* pos_ctx, int B, int L, int b, int a, const CacheView& c,
                                    int32_t* aug_pos, int32_t* block_map, cudaStream_t st);
@@ -61,6 +74,7 @@ struct AttnLaunch {
   float* lse_f32;         // mode 1: [parts][B][T][Hq]
   int chunks_per_block;   // mode 1
   int anchor;             // mode 0: anchor size a (the first a keys of block 1)
+  SeqShift shift;         // per-sequence context lengths L + delta[s] (on = 0: all L)
   const void* anchor_k;   // mode 0: NULL (anchor keys are block 1's cached keys) or bf16 [B][n-1][Hkv][a][d]
   float scale_log2;
   RopeTable rope;
@@ -75,7 +89,8 @@ struct DecodeLaunch {
   const void* k_new;      // [B][Hkv][d] bf16 (pre-RoPE): appended at slot n_keys - 1 by the kernel
   const void* v_new;      // [B][Hkv][d] bf16
   const int32_t* pos;     // [B] position of the decoded token
-  int n_keys;             // keys [0, n_keys) of every sequence
+  int n_keys;             // keys [0, n_keys) of every sequence (the longest, with a shift)
+  SeqShift shift;         // sequence s has n_keys + delta[s] keys
   int chunk;              // keys per CTA
   CacheView cache;
   float* o_ws;            // [nchunks][B*Hq][d]

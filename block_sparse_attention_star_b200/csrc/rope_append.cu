@@ -22,6 +22,8 @@
 #include "common.cuh"
 #include "internal.h"
 
+#include <algorithm>
+
 namespace star {
 namespace {
 
@@ -36,7 +38,8 @@ __global__ void __launch_bounds__(256) rope_append_kernel(const bf16* __restrict
                                                           const int32_t* __restrict__ pos, int B, int ntok, int start,
                                                           int Hkv, bf16* __restrict__ kpool, bf16* __restrict__ vpool,
                                                           const int32_t* __restrict__ page_table, int max_pages,
-                                                          int num_pages, int P, const __grid_constant__ RopeParams rp) {
+                                                          int num_pages, int P, const __grid_constant__ RopeParams rp,
+                                                          const __grid_constant__ SeqShift sh) {
   constexpr int CH = D / 16;
   const long long total = (long long)B * ntok * CH;
   for (long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x; gid < total;
@@ -45,7 +48,7 @@ __global__ void __launch_bounds__(256) rope_append_kernel(const bf16* __restrict
     const long long r = gid / CH;
     const int t = (int)(r % ntok);
     const int bi = (int)(r / ntok);
-    const int slot_abs = start + t;
+    const int slot_abs = start + (sh.on ? sh.delta[bi] : 0) + t;
     const int page = page_table[(size_t)bi * max_pages + slot_abs / P];
     if (page < 0 || page >= num_pages) {
       record_error(kDevBadPage);
@@ -152,8 +155,10 @@ __global__ void __launch_bounds__(256) rope_anchor_kernel(const bf16* __restrict
   }
 }
 
+// Slots [from + delta[bi], to) of every sequence bi; `from` is the smallest start over the batch.
 __global__ void zero_slots_kernel(int B, int from, int to, int Hkv, int d, bf16* kpool, bf16* vpool,
-                                  const int32_t* page_table, int max_pages, int num_pages, int P) {
+                                  const int32_t* page_table, int max_pages, int num_pages, int P,
+                                  const __grid_constant__ SeqShift sh, int from_cap) {
   const int CH = d / 8;
   const long long span = to - from;
   const long long total = (long long)B * span * Hkv * CH;
@@ -165,6 +170,7 @@ __global__ void zero_slots_kernel(int B, int from, int to, int Hkv, int d, bf16*
     r /= Hkv;
     const int s = from + (int)(r % span);
     const int bi = (int)(r / span);
+    if (sh.on && s < from_cap + sh.delta[bi]) continue;  // still this sequence's context
     const int page = page_table[(size_t)bi * max_pages + s / P];
     if (page < 0 || page >= num_pages) {
       record_error(kDevBadPage);
@@ -221,8 +227,11 @@ int grid_for(long long work, int threads) {
 cudaError_t read_and_clear_error_rope(int* code) { return read_and_clear_tu_error(code); }
 
 cudaError_t launch_rope_append(const void* k, const void* v, const int32_t* pos, int B, int ntok, int start, int Hkv,
-                               int d, const CacheView& c, const RopeTable& rt, cudaStream_t st) {
+                               int d, const CacheView& c, const RopeTable& rt, cudaStream_t st, const SeqShift* shift) {
   if (ntok <= 0 || B <= 0) return cudaSuccess;
+  SeqShift sh;
+  sh.on = 0;
+  if (shift && shift->on) sh = *shift;
   RopeParams rp;
   for (int j = 0; j < d / 2; ++j) rp.inv_freq[j] = rt.inv_freq[j];
   const long long work = (long long)B * ntok * (d / 16);
@@ -231,12 +240,12 @@ cudaError_t launch_rope_append(const void* k, const void* v, const int32_t* pos,
     rope_append_kernel<128><<<grid, 256, 0, st>>>(
         reinterpret_cast<const bf16*>(k), reinterpret_cast<const bf16*>(v), pos, B, ntok, start, Hkv,
         reinterpret_cast<bf16*>(c.k_pool), reinterpret_cast<bf16*>(c.v_pool), c.page_table, c.max_pages,
-        c.num_pages, c.P, rp);
+        c.num_pages, c.P, rp, sh);
   } else {
     rope_append_kernel<64><<<grid, 256, 0, st>>>(
         reinterpret_cast<const bf16*>(k), reinterpret_cast<const bf16*>(v), pos, B, ntok, start, Hkv,
         reinterpret_cast<bf16*>(c.k_pool), reinterpret_cast<bf16*>(c.v_pool), c.page_table, c.max_pages,
-        c.num_pages, c.P, rp);
+        c.num_pages, c.P, rp, sh);
   }
   return cudaGetLastError();
 }
@@ -257,12 +266,20 @@ cudaError_t launch_rope_q(const void* q, const int32_t* pos, int B, int ntok, in
   return cudaGetLastError();
 }
 
-cudaError_t launch_zero_slots(int B, int from, int to, int Hkv, int d, const CacheView& c, cudaStream_t st) {
-  if (to <= from) return cudaSuccess;
-  const long long work = (long long)B * (to - from) * Hkv * (d / 8);
-  zero_slots_kernel<<<grid_for(work, 256), 256, 0, st>>>(B, from, to, Hkv, d, reinterpret_cast<bf16*>(c.k_pool),
+cudaError_t launch_zero_slots(int B, int from, int to, int Hkv, int d, const CacheView& c, cudaStream_t st,
+                              const SeqShift* shift) {
+  SeqShift sh;
+  sh.on = 0;
+  int lo = from;
+  if (shift && shift->on) {
+    sh = *shift;
+    for (int i = 0; i < B; ++i) lo = std::min(lo, from + sh.delta[i]);
+  }
+  if (to <= lo) return cudaSuccess;
+  const long long work = (long long)B * (to - lo) * Hkv * (d / 8);
+  zero_slots_kernel<<<grid_for(work, 256), 256, 0, st>>>(B, lo, to, Hkv, d, reinterpret_cast<bf16*>(c.k_pool),
                                                           reinterpret_cast<bf16*>(c.v_pool), c.page_table,
-                                                          c.max_pages, c.num_pages, c.P);
+                                                          c.max_pages, c.num_pages, c.P, sh, from);
   return cudaGetLastError();
 }
 

@@ -72,6 +72,17 @@ typedef struct star_shape {
   int32_t anchor;      /* anchor size a: the first a tokens of block 1 ("仓库里的真实实现":
                           anchor_block_size is a parameter of its own); 0 means b (the pages'
                           default, the whole first block); a multiple of 128 and <= b */
+  const int32_t* seq_len; /* HOST int32 [B] or NULL: per-sequence context lengths L_s, 1 <= L_s <= L
+                          (B <= 256).  L is then the capacity (a multiple of b); sequence s has
+                          ceil(L_s / b) blocks, the last one ragged ("问题定义与记号" splits the
+                          context into blocks of b tokens; an uneven split ends in a short
+                          block), and its tail (query and generated tokens) starts at L_s.
+                          Context arrays stay padded to L; rows >= L_s of outputs are
+                          unspecified.  Cache indices given to star_kv_append (start) and
+                          star_decode_step (cur_len) are in the frame of a sequence of length
+                          L: sequence s uses index + L_s - L, so they must be >= L.
+                          Phase-2 partials of blocks a sequence does not have are empty
+                          (O = 0, LSE = -inf), which star_lse_merge skips. */
 } star_shape;
 
 /* Paged KV cache ("局部注意力与 KV 丢弃": only non-anchor KV is kept).

@@ -34,6 +34,7 @@ class Workload:
     anchor: int = 0                 # anchor size a (the first a tokens of block 1); 0 = b
     anchor_ids: str = "context"     # anchor position ids: "context" (tokens 0..a-1's own),
                                     # "offset" (per block, a seeded offset inside the prefix), "zero"
+    seq_lens: tuple | None = None   # per-sequence context lengths (<= L, the capacity); None = all L
 
     @property
     def a(self) -> int:
@@ -72,6 +73,9 @@ class Workload:
 
     def phase1_flops(self) -> float:
         return 4.0 * self.d * self.Hq * self.B * self.phase1_pairs_per_head()
+
+    def ctx_len(self, bi: int) -> int:
+        return self.seq_lens[bi] if self.seq_lens is not None else self.L
 
     def kv_bytes(self, tokens: int) -> int:
         """bf16 K plus V bytes for ``tokens`` cached tokens of every sequence."""

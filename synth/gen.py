@@ -173,14 +173,18 @@ def make_inputs(wl: Workload, device="cpu", parts=("ctx", "query", "dec")) -> di
         g["pos_ctx"] = torch.arange(L, dtype=torch.int32, device=device).repeat(B, 1).contiguous()
         if wl.anchor_ids != "context" and wl.n > 1:
             g["anchor_pos"] = anchor_positions(wl, device)
+    # Each sequence's query and generated tokens follow its own context.
+    ends = torch.tensor([wl.ctx_len(bi) for bi in range(B)], dtype=torch.int32, device=device)
+    if wl.seq_lens is not None:
+        g["seq_len"] = ends.clone()
     if "query" in parts:
         g["q_query"] = gaussian_bf16(wl.seed, STREAM_IDS["q_query"], (B, T, Hq, d), device)
         g["k_query"] = gaussian_bf16(wl.seed, STREAM_IDS["k_query"], (B, T, Hkv, d), device)
         g["v_query"] = gaussian_bf16(wl.seed, STREAM_IDS["v_query"], (B, T, Hkv, d), device)
-        g["pos_query"] = (L + torch.arange(T, dtype=torch.int32, device=device)).repeat(B, 1).contiguous()
+        g["pos_query"] = (ends[:, None] + torch.arange(T, dtype=torch.int32, device=device)[None, :]).contiguous()
     if "dec" in parts:
         g["q_dec"] = gaussian_bf16(wl.seed, STREAM_IDS["q_dec"], (S, B, 1, Hq, d), device)
         g["k_dec"] = gaussian_bf16(wl.seed, STREAM_IDS["k_dec"], (S, B, 1, Hkv, d), device)
         g["v_dec"] = gaussian_bf16(wl.seed, STREAM_IDS["v_dec"], (S, B, 1, Hkv, d), device)
-        g["pos_dec"] = (L + T + torch.arange(S, dtype=torch.int32, device=device)).unsqueeze(1).repeat(1, B).contiguous()
+        g["pos_dec"] = (T + torch.arange(S, dtype=torch.int32, device=device)[:, None] + ends[None, :]).contiguous()
     return g

@@ -23,7 +23,8 @@ LSE_ABS = 1e-3
 
 def shape_of(wl: Workload) -> star.StarShape:
     return star.StarShape.make(B=wl.B, Hq=wl.Hq, Hkv=wl.Hkv, d=wl.d, L=wl.L, b=wl.b, T_max=wl.T_max,
-                               page_tokens=wl.page_tokens, rope_theta=wl.theta, anchor=wl.anchor)
+                               page_tokens=wl.page_tokens, rope_theta=wl.theta, anchor=wl.anchor,
+                               seq_len=wl.seq_lens)
 
 
 def to64(t: torch.Tensor) -> np.ndarray:
@@ -83,9 +84,14 @@ class Err:
 
 
 def err(gpu, ref) -> Err:
+    """Max and mean abs difference; where the oracle has -inf (an empty partial's LSE)
+    the GPU value must be -inf too, and those elements are left out of the statistics."""
     g = to64(gpu) if isinstance(gpu, torch.Tensor) else np.asarray(gpu, dtype=np.float64)
     r = np.asarray(ref, dtype=np.float64)
     assert g.shape == r.shape, (g.shape, r.shape)
+    empty = np.isneginf(r)
+    assert np.array_equal(np.isneginf(g), empty), "-inf (empty partial) pattern differs"
+    g, r = g[~empty], r[~empty]
     d = np.abs(g - r)
     return Err(float(d.max()) if d.size else 0.0, float(d.mean()) if d.size else 0.0)
 
@@ -107,6 +113,7 @@ def assert_out(gpu, ref, what: str):
     e = err(gpu, ref)
     g = to64(gpu) if isinstance(gpu, torch.Tensor) else np.asarray(gpu, dtype=np.float64)
     r = np.asarray(ref, dtype=np.float64)
+    assert np.all(np.isfinite(g)), f"{what}: non-finite output"
     bound = np.maximum(MAX_ABS, 0.5 * bf16_spacing(r) + 4e-3)
     over = np.abs(g - r) > bound
     worst = np.unravel_index(np.argmax(np.abs(g - r) - bound), r.shape) if r.size else None
