@@ -25,6 +25,7 @@ import json
 import os
 import statistics
 import subprocess
+import threading
 import sys
 import time
 
@@ -83,21 +84,41 @@ class ClockSampler:
                     "--format=csv,noheader,nounits", "-lms", "50"]
 
     def __enter__(self):
+        """Start nvidia-smi and return once it has produced its first sample, so that the timed
+        region that follows is covered from its start."""
+        self.samples = []
         try:
             self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
+            return self
+
+        def read():
+            for ln in self.proc.stdout:
+                if ln.strip():
+                    self.samples.append((time.monotonic(), ln))
+
+        self.reader = threading.Thread(target=read, daemon=True)
+        self.reader.start()
+        deadline = time.monotonic() + 5.0
+        while not self.samples and time.monotonic() < deadline:
+            time.sleep(0.01)
+        self.t0 = time.monotonic()
         return self
 
     def __exit__(self, *exc):
+        t1 = time.monotonic()
         if self.proc is not None:
+            time.sleep(0.06)  # the sample that closes the window
             self.proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+            self.reader.join(timeout=5)
+            inside = [ln for t, ln in self.samples if self.t0 <= t <= t1 + 0.06]
+            after = [ln for t, ln in self.samples if t >= self.t0]
+            self.lines = inside or after[:1]
 
     def summary(self):
         sm, smax, reasons = [], [], set()
