@@ -226,9 +226,9 @@ def max_over_ranks(value: float, device) -> float:
     return float(t.item())
 
 
-def job_value(world: int, B: int, L: int, ms_per_step: float) -> float:
-    """Whole-job context tokens per second: every rank encodes B sequences of L tokens per step."""
-    return world * B * L / (ms_per_step * 1e-3)
+def job_value(world: int, ctx_tokens: int, ms_per_step: float) -> float:
+    """Whole-job context tokens per second: every rank encodes its batch's context each step."""
+    return world * ctx_tokens / (ms_per_step * 1e-3)
 
 
 def _ev():
@@ -315,24 +315,24 @@ def run_star(args, rank, world, local_rank):
     dec_call_ms = [e["dec_call"][s][0].elapsed_time(e["dec_call"][s][1]) for e in evs for s in range(wl.S)]
     flops = wl.phase1_flops()
     tflops = flops / (p1_ms * 1e-3) / 1e12
-    dec_bytes = statistics.mean(wl.kv_bytes(wl.L + wl.T + s + 1) for s in range(wl.S))
+    dec_bytes = statistics.mean(wl.decode_bytes(s) for s in range(wl.S))
     dec_gbs = dec_bytes / (statistics.mean(dec_kernel_ms) * 1e-3) / 1e9
 
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(run, K, max(3, args.warmup), world)
 
-    value = job_value(world, wl.B, wl.L, ms_step)
+    value = job_value(world, wl.context_tokens(), ms_step)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": max(3, args.warmup),
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16; 1% of context key rows x8 where the workload says peaky)",
         "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d, "L": wl.L, "b": wl.b,
                    "n": wl.n, "T": wl.T, "S": wl.S, "page_tokens": wl.page_tokens, "anchor": wl.a,
-                   "anchor_ids": wl.anchor_ids,
+                   "anchor_ids": wl.anchor_ids, "seq_lens": list(wl.seq_lens) if wl.seq_lens else None,
                    "parallelism": f"independent sequences per GPU x{world}",
                    "l2": "inputs larger than L2 (no flush)"},
-        "phase1": {"attn_ms": p1_ms, "ctx_tok_s": wl.B * wl.L / (p1_ms * 1e-3), "tflops": tflops,
+        "phase1": {"attn_ms": p1_ms, "ctx_tok_s": wl.context_tokens() / (p1_ms * 1e-3), "tflops": tflops,
                    "frac_bf16_burst": tflops / peaks["bf16"], "frac_bf16_sustained": tflops / peaks["bf16_sustained"]},
         "phase2": {"attn_ms": p2_ms},
         "decode": {"us_per_step": 1e3 * statistics.mean(dec_call_ms), "kernel_us": 1e3 * statistics.mean(dec_kernel_ms),
@@ -426,7 +426,7 @@ def run_e2e(run, K, W, world):
     torch.cuda.synchronize()
     use(0)
     ms = max_over_ranks(t0.elapsed_time(t1) / K, run.dev)
-    return {"value": job_value(world, wl.B, wl.L, ms), "unit": UNIT,
+    return {"value": job_value(world, wl.context_tokens(), ms), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
             "copies": "pipelined: step k+1's inputs upload and step k's results download while step k computes"}
 

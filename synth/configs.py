@@ -71,8 +71,24 @@ class Workload:
         tri = b * (b + 1) // 2
         return tri + (n - 1) * (a * b + tri)
 
+    def phase1_pairs_of(self, length: int) -> int:
+        """Pairs of one head of a sequence of ``length`` context tokens (the last block
+        ragged when b does not divide it)."""
+        b, a = self.b, self.a
+        total = 0
+        for i in range(-(-length // b)):
+            n_i = min(b, length - i * b)
+            total += n_i * (n_i + 1) // 2 + (a * n_i if i > 0 else 0)
+        return total
+
+    def context_tokens(self) -> int:
+        """Context tokens of the whole batch."""
+        return sum(self.ctx_len(bi) for bi in range(self.B))
+
     def phase1_flops(self) -> float:
-        return 4.0 * self.d * self.Hq * self.B * self.phase1_pairs_per_head()
+        if self.seq_lens is None:
+            return 4.0 * self.d * self.Hq * self.B * self.phase1_pairs_per_head()
+        return 4.0 * self.d * self.Hq * sum(self.phase1_pairs_of(self.ctx_len(bi)) for bi in range(self.B))
 
     def ctx_len(self, bi: int) -> int:
         return self.seq_lens[bi] if self.seq_lens is not None else self.L
@@ -80,6 +96,11 @@ class Workload:
     def kv_bytes(self, tokens: int) -> int:
         """bf16 K plus V bytes for ``tokens`` cached tokens of every sequence."""
         return tokens * self.Hkv * self.d * 2 * 2 * self.B
+
+    def decode_bytes(self, step: int) -> int:
+        """K and V bytes one decode step reads: every sequence's context, query tail, the
+        tokens generated before and the new one."""
+        return sum(self.ctx_len(bi) + self.T + step + 1 for bi in range(self.B)) * self.Hkv * self.d * 2 * 2
 
 
 _BASE = {
@@ -104,6 +125,9 @@ CONFIGS: dict[str, Workload] = {
                                                             anchor=8192, anchor_ids="offset"),
     "llama8b-128k-b32768-zero": dataclasses.replace(_BASE["llama8b-128k"], name="llama8b-128k-b32768-zero",
                                                     anchor_ids="zero"),
+    # variable-length batch: a full 128K context beside a 100000-token one (ragged seventh block)
+    "llama70b-128k-var": dataclasses.replace(_BASE["llama70b-128k"], name="llama70b-128k-var",
+                                             seq_lens=(131072, 100000)),
 }
 
 

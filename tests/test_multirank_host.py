@@ -34,7 +34,7 @@ def _worker(rank, world, port, q):
         from synth import make_inputs
         tiny = bench.rank_workload("tiny", rank)
         x = make_inputs(tiny, "cpu", parts=("query",))["q_query"].float().sum().item()
-        q.put((rank, wl.seed, slowest, bench.job_value(world, wl.B, wl.L, slowest), x))
+        q.put((rank, wl.seed, slowest, bench.job_value(world, wl.context_tokens(), slowest), x))
     finally:
         dist.destroy_process_group()
 
