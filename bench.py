@@ -143,6 +143,14 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # The CUDA path
 # ---------------------------------------------------------------------------
+def workload_shape(wl):
+    """The C-ABI shape of a workload: sizes, anchor and per-sequence context lengths."""
+    import block_sparse_attention_star_b200 as star
+    return star.StarShape.make(B=wl.B, Hq=wl.Hq, Hkv=wl.Hkv, d=wl.d, L=wl.L, b=wl.b, T_max=wl.T_max,
+                               page_tokens=wl.page_tokens, rope_theta=wl.theta, anchor=wl.anchor,
+                               seq_len=wl.seq_lens)
+
+
 class StarRun:
     """Buffers and the step sequence of one workload on one GPU."""
 
@@ -150,8 +158,7 @@ class StarRun:
         import block_sparse_attention_star_b200 as star
         self.star, self.wl, self.dev = star, wl, device
         self.inp = make_inputs(wl, device)
-        self.shape = star.StarShape.make(B=wl.B, Hq=wl.Hq, Hkv=wl.Hkv, d=wl.d, L=wl.L, b=wl.b, T_max=wl.T_max,
-                                         page_tokens=wl.page_tokens, rope_theta=wl.theta, anchor=wl.anchor)
+        self.shape = workload_shape(wl)
         self.cache = star.PagedKVCache(self.shape, device=device)
         self.o_ctx = torch.empty_like(self.inp["q_ctx"])
         self.o_part, self.lse_part = star.alloc_partials(self.shape, wl.T, device)

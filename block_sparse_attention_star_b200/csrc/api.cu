@@ -444,11 +444,19 @@ int star_decode_step(const star_shape* shape, const star_cache* cache, const voi
   const star::CacheView cv = view(shape, cache);
   const star::RopeTable rt = rope_table(shape);
   cudaError_t e;
-  const int chunk = decode_chunk(shape);
+  // The workspace holds the chunks of the capacity at the capacity's chunk; per-sequence
+  // lengths may take a longer chunk (never a shorter one) to balance the real work.
+  const int chunk_cap = decode_chunk(shape);
   const int n_keys = cur_len + 1;
+  int chunk = chunk_cap;
+  if (shape->seq_len) {
+    int keys_of[star::kMaxVarB];
+    for (int s = 0; s < shape->B; ++s) keys_of[s] = n_keys + shape->seq_len[s] - shape->L;
+    chunk = star::decode_pick_chunk_var(shape->B, shape->Hkv, keys_of, chunk_cap, num_sms());
+  }
   const int nch = star::decode_num_chunks(n_keys, chunk);
   const size_t rows = (size_t)shape->B * shape->Hq;
-  const size_t nch_max = (size_t)star::decode_num_chunks(shape->L + shape->T_max, chunk);
+  const size_t nch_max = (size_t)star::decode_num_chunks(shape->L + shape->T_max, chunk_cap);
   star::DecodeLaunch a;
   a.B = shape->B;
   a.Hq = shape->Hq;

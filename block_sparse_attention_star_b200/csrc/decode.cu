@@ -67,6 +67,12 @@ struct DecParams {
   int item_base, num_items;  // this launch: items [item_base, num_items)
   float scale_log2;
   SeqShift sh;               // sequence bi has n_keys + delta[bi] keys (sh.on = 0: all n_keys)
+  // sh.on: the item space lists every sequence's non-empty chunks first (sequence bi's
+  // at [item_off[bi], item_off[bi+1]), head-major, chunk fastest), then the empty chunk
+  // slots past the shorter sequences ([item_off[B] + empty_off[bi], ...)), so that the
+  // round-robin assignment spreads the real work evenly over the CTAs.
+  int item_off[kMaxVarB + 1];
+  int empty_off[kMaxVarB + 1];
   double inv_freq[kMaxHalfDim];
 };
 
@@ -96,11 +102,37 @@ struct DecItem {
   int last;    // the chunk holds the sequence's last key (the new token's slot)
 };
 
+// The last sequence s in [0, B) with off[s] <= x (off is non-decreasing, off[0] = 0 <= x).
+__device__ __forceinline__ int seq_of(const int* off, int B, int x) {
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (off[mid] <= x) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
 __device__ __forceinline__ DecItem dec_item(const DecParams& p, int idx) {
   DecItem it;
-  it.c = idx % p.nchunks;
-  it.g = (idx / p.nchunks) % p.Hkv;
-  it.bi = idx / (p.nchunks * p.Hkv);
+  if (!p.sh.on) {
+    it.c = idx % p.nchunks;
+    it.g = (idx / p.nchunks) % p.Hkv;
+    it.bi = idx / (p.nchunks * p.Hkv);
+  } else if (idx < p.item_off[p.B]) {
+    it.bi = seq_of(p.item_off, p.B, idx);
+    const int w = idx - p.item_off[it.bi];
+    const int nc = (p.item_off[it.bi + 1] - p.item_off[it.bi]) / p.Hkv;
+    it.g = w / nc;
+    it.c = w - it.g * nc;
+  } else {
+    const int e = idx - p.item_off[p.B];
+    it.bi = seq_of(p.empty_off, p.B, e);
+    const int w = e - p.empty_off[it.bi];
+    const int ne = (p.empty_off[it.bi + 1] - p.empty_off[it.bi]) / p.Hkv;
+    it.g = w / ne;
+    it.c = p.nchunks - ne + (w - it.g * ne);
+  }
   it.n_keys = p.n_keys + (p.sh.on ? p.sh.delta[it.bi] : 0);
   it.k_begin = it.c * p.chunk;
   it.k_end = min(it.k_begin + p.chunk, it.n_keys);
@@ -564,6 +596,28 @@ cudaError_t read_and_clear_error_decode(int* code) { return read_and_clear_tu_er
 
 int decode_num_chunks(int n_keys, int chunk) { return (n_keys + chunk - 1) / chunk; }
 
+// Per-sequence key counts: the chunk (at least min_chunk keys, a multiple of 128) that
+// minimises the tiles of the busiest CTA over the non-empty items, with the same quarter
+// tile of overhead per item as the uniform choice.
+int decode_pick_chunk_var(int B, int Hkv, const int* n_keys_of, int min_chunk, int num_sms) {
+  long long tmax = 1;
+  for (int s = 0; s < B; ++s) tmax = std::max<long long>(tmax, (n_keys_of[s] + kTileKeys - 1) / kTileKeys);
+  const long long ct_min = std::max(1, min_chunk / kTileKeys);
+  long long best_ct = std::max(ct_min, tmax), best_cost = -1;
+  for (long long ct = ct_min; ct <= tmax; ++ct) {
+    long long items = 0;
+    for (int s = 0; s < B; ++s) items += (long long)Hkv * ((n_keys_of[s] + ct * kTileKeys - 1) / (ct * kTileKeys));
+    const long long ctas = std::min<long long>(items, num_sms);
+    const long long per = (items + ctas - 1) / ctas;
+    const long long cost = 4 * per * ct + per;
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best_ct = ct;
+    }
+  }
+  return (int)(best_ct * kTileKeys);
+}
+
 // Keys per chunk (a multiple of the 128-key tile) for caches of up to n_keys keys:
 // the chunk count that minimises the tiles of the busiest CTA, counting each item
 // a quarter tile of overhead.
@@ -620,6 +674,17 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t st) {
   p.sh = a.shift;
   for (int j = 0; j < kMaxHalfDim; ++j) p.inv_freq[j] = j < a.d / 2 ? a.rope.inv_freq[j] : 0.0;
   if (a.chunk <= 0 || a.chunk % kTileKeys != 0 || a.cache.P % kTileKeys != 0) return cudaErrorInvalidValue;
+  p.item_off[0] = p.empty_off[0] = 0;
+  if (p.sh.on) {
+    if (a.B > kMaxVarB) return cudaErrorInvalidValue;
+    for (int s = 0; s < a.B; ++s) {
+      const int ks = a.n_keys + p.sh.delta[s];
+      if (ks < 1 || ks > a.n_keys) return cudaErrorInvalidValue;
+      const int nc = decode_num_chunks(ks, a.chunk);
+      p.item_off[s + 1] = p.item_off[s] + a.Hkv * nc;
+      p.empty_off[s + 1] = p.empty_off[s] + a.Hkv * (p.nchunks - nc);
+    }
+  }
   CUtensorMap mk, mv;
   if (!make_tile_map(&mk, a.cache.k_pool, a.d, a.cache.P, a.Hkv, a.cache.num_pages) ||
       !make_tile_map(&mv, a.cache.v_pool, a.d, a.cache.P, a.Hkv, a.cache.num_pages))

@@ -51,6 +51,8 @@ def run_gpu(wl: Workload, inp: dict, page_table: torch.Tensor | None = None, num
         T = wl.T
         o_part, lse_part = star.alloc_partials(shape, T, dev)
         ws = star.workspace(shape, star.STAR_OP_PHASE2, T, dev)
+        for t in (o_part, lse_part, ws):  # NaN bytes: a slot the kernels leave unwritten shows up
+            t.view(torch.uint8).fill_(0xFF)
         star.star_phase2_partial(shape, cache, inp["q_query"], inp["k_query"], inp["v_query"], inp["pos_query"], T,
                                  o_part, lse_part, ws)
         o_q = torch.empty((wl.B, T, wl.Hq, wl.d), dtype=torch.bfloat16, device=dev)
@@ -59,6 +61,7 @@ def run_gpu(wl: Workload, inp: dict, page_table: torch.Tensor | None = None, num
         res.update(o_part=o_part, lse_part=lse_part, o_query=o_q, lse_query=lse_q)
     if "decode" in phases:
         wsd = star.workspace(shape, star.STAR_OP_DECODE, 0, dev)
+        wsd.fill_(0xFF)
         o_dec = torch.empty((wl.S, wl.B, 1, wl.Hq, wl.d), dtype=torch.bfloat16, device=dev)
         lse_dec = torch.empty((wl.S, wl.B, wl.Hq), dtype=torch.float32, device=dev)
         for s in range(wl.S):

@@ -65,6 +65,19 @@ def test_workspace_sizes_for_every_workload():
             star.star_workspace_size(sh, star.STAR_OP_PHASE2, wl.T_max + 1)
 
 
+def test_bench_shape_carries_every_workload_field():
+    """The timed shape is the workload's: anchor and per-sequence context lengths included."""
+    import bench
+    for wl in CONFIGS.values():
+        sh = bench.workload_shape(wl)
+        assert (sh.B, sh.Hq, sh.Hkv, sh.d, sh.L, sh.b, sh.T_max) == (wl.B, wl.Hq, wl.Hkv, wl.d, wl.L, wl.b, wl.T_max)
+        assert sh.anchor == (wl.anchor or 0)
+        if wl.seq_lens is None:
+            assert not sh.seq_len
+        else:
+            assert [sh.seq_len[i] for i in range(wl.B)] == list(wl.seq_lens)
+
+
 def test_anchor_workspace_size():
     """The anchor's keys roped at caller ids: bf16 [B][n-1][Hkv][a][d]; a = b when the shape says 0."""
     for a in (0, 8192, 32768):
