@@ -176,7 +176,7 @@ class StarRun:
     def step(self, ev=None):
         """One pass of the hot path.  ev: optional dict of (start, stop) event lists to record."""
         s, wl, inp = self.star, self.wl, self.inp
-        if ev:
+        if ev and "p1" in ev:
             s.star_set_trace_events(*ev["p1"])
         if self.ws1 is not None:
             s.star_phase1_encode_anchored(self.shape, self.cache, inp["q_ctx"], inp["k_ctx"], inp["v_ctx"],
@@ -184,21 +184,24 @@ class StarRun:
         else:
             s.star_phase1_encode(self.shape, self.cache, inp["q_ctx"], inp["k_ctx"], inp["v_ctx"], inp["pos_ctx"],
                                  self.o_ctx)
-        if ev:
+        if ev and "p2" in ev:
             s.star_set_trace_events(*ev["p2"])
         s.star_phase2_partial(self.shape, self.cache, inp["q_query"], inp["k_query"], inp["v_query"], inp["pos_query"],
                               wl.T, self.o_part, self.lse_part, self.ws2)
         if ev:
             s.star_set_trace_events(None, None)
         s.star_lse_merge(self.shape.n, wl.B * wl.T * wl.Hq, wl.d, self.o_part, self.lse_part, self.o_q, self.lse_q)
+        # ev["dec_span"] brackets the S decode steps with nothing between their launches;
+        # ev["dec"] (a separate instrumented step) brackets every decode attention kernel.
+        if ev and "dec_span" in ev:
+            ev["dec_span"][0].record()
         for st in range(wl.S):
-            if ev:
+            if ev and "dec" in ev:
                 s.star_set_trace_events(*ev["dec"][st])
-                ev["dec_call"][st][0].record()
             s.star_decode_step(self.shape, self.cache, inp["q_dec"][st], inp["k_dec"][st], inp["v_dec"][st],
                                inp["pos_dec"][st], wl.L + wl.T + st, self.o_dec[st], self.lse_dec[st], self.wsd)
-            if ev:
-                ev["dec_call"][st][1].record()
+        if ev and "dec_span" in ev:
+            ev["dec_span"][1].record()
         if ev:
             s.star_set_trace_events(None, None)
 
@@ -299,8 +302,7 @@ def run_star(args, rank, world, local_rank):
         raise RuntimeError("device error after warm-up")
 
     K = args.steps
-    evs = [{"p1": _pair(), "p2": _pair(), "dec": [_pair() for _ in range(wl.S)],
-            "dec_call": [_tpair() for _ in range(wl.S)]} for _ in range(K)]
+    evs = [{"p1": _pair(), "p2": _pair(), "dec_span": _tpair()} for _ in range(K)]
     t0, t1 = _ev(), _ev()
     if world > 1:
         dist.barrier()
@@ -315,11 +317,15 @@ def run_star(args, rank, world, local_rank):
         dist.barrier()
     status = star.star_device_status()
     ms_step = max_over_ranks(t0.elapsed_time(t1), dev) / K
+    # The decode attention kernel alone: one more (untimed) step with events around each launch.
+    ev_dec = {"dec": [_pair() for _ in range(wl.S)]}
+    run.step(ev_dec)
+    torch.cuda.synchronize()
 
     p1_ms = statistics.mean(e["p1"][0].elapsed_time(e["p1"][1]) for e in evs)
     p2_ms = statistics.mean(e["p2"][0].elapsed_time(e["p2"][1]) for e in evs)
-    dec_kernel_ms = [e["dec"][s][0].elapsed_time(e["dec"][s][1]) for e in evs for s in range(wl.S)]
-    dec_call_ms = [e["dec_call"][s][0].elapsed_time(e["dec_call"][s][1]) for e in evs for s in range(wl.S)]
+    dec_kernel_ms = [ev_dec["dec"][s][0].elapsed_time(ev_dec["dec"][s][1]) for s in range(wl.S)]
+    dec_step_ms = statistics.mean(e["dec_span"][0].elapsed_time(e["dec_span"][1]) for e in evs) / wl.S
     flops = wl.phase1_flops()
     tflops = flops / (p1_ms * 1e-3) / 1e12
     dec_bytes = statistics.mean(wl.decode_bytes(s) for s in range(wl.S))
@@ -342,8 +348,11 @@ def run_star(args, rank, world, local_rank):
         "phase1": {"attn_ms": p1_ms, "ctx_tok_s": wl.context_tokens() / (p1_ms * 1e-3), "tflops": tflops,
                    "frac_bf16_burst": tflops / peaks["bf16"], "frac_bf16_sustained": tflops / peaks["bf16_sustained"]},
         "phase2": {"attn_ms": p2_ms},
-        "decode": {"us_per_step": 1e3 * statistics.mean(dec_call_ms), "kernel_us": 1e3 * statistics.mean(dec_kernel_ms),
-                   "bytes_per_step": dec_bytes, "kernel_gbs": dec_gbs, "frac_hbm": dec_gbs / peaks["hbm_gbs"]},
+        "decode": {"us_per_step": 1e3 * dec_step_ms, "kernel_us": 1e3 * statistics.mean(dec_kernel_ms),
+                   "bytes_per_step": dec_bytes, "kernel_gbs": dec_gbs, "frac_hbm": dec_gbs / peaks["hbm_gbs"],
+                   "step_gbs": dec_bytes / (dec_step_ms * 1e-3) / 1e9,
+                   "timing": "us_per_step: the S steps' span in the timed region / S (append, attention, merge "
+                             "and launch gaps); kernel_us: the attention kernel alone, one extra untimed step"},
         "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
                      "frac": tflops / peaks["bf16_sustained"], "traffic": measured_traffic(wl.B, wl.L),
                      "kernel": f"star_attn_kernel<{wl.d},0> (Phase 1)", "flop_per_launch": flops,

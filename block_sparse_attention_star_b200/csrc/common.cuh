@@ -141,6 +141,16 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the previous kernel in the stream drains; it runs
+// its prologue, then griddep_wait() blocks until that kernel has completed and its
+// writes are visible (a no-op for a normal launch).  griddep_launch_dependents()
+// lets the next such kernel be scheduled before this one ends.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------
 // tcgen05 (1-CTA group)
 // ---------------------------------------------------------------------------

@@ -238,6 +238,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // q and P operands: the padding rows (heads G..15) are zeros.
   for (int i = threadIdx.x; i < (S::kXch - S::kQ) / 16; i += kThreads)
     reinterpret_cast<uint4*>(smem + S::kQ)[i] = make_uint4(0u, 0u, 0u, 0u);
+  // Everything above touches only this CTA's on-chip state, so it overlaps the
+  // previous kernel's tail; global memory is read and written only after it ends.
+  griddep_wait();
+  griddep_launch_dependents();
   __syncthreads();
 
   for (int ii = 0; ii < n_my; ++ii) {
@@ -583,8 +587,7 @@ cudaError_t launch_dg(DecParams p, const CUtensorMap& mk, const CUtensorMap& mv,
   for (int base = 0; base < total_items; base += grid * kMaxItems) {
     p.item_base = base;
     p.num_items = std::min(total_items, base + grid * kMaxItems);
-    kern<<<std::min(grid, p.num_items - base), kThreads, S::kBytes, st>>>(mk, mv, p);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(kern, std::min(grid, p.num_items - base), kThreads, S::kBytes, st, mk, mv, p);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

@@ -5,7 +5,28 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace star {
+
+// A launch with programmatic stream serialization: the kernel may start while the
+// previous kernel in the stream drains, and waits (griddepcontrol.wait) before it
+// touches global memory.
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 constexpr int kMaxHalfDimHost = 64;
 constexpr int kMaxVarB = 256;   // sequences of a batch with per-sequence lengths (passed by value)

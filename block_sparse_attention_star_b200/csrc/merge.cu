@@ -48,6 +48,8 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(int parts_per_group, lon
                                                         float* __restrict__ lse_out) {
   constexpr int PER = D / 32;
   using V = typename Cols<D>::T;
+  griddep_wait();  // the partials come from the previous kernel
+  griddep_launch_dependents();
   const int lane = threadIdx.x % 32;
   const long long row = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
   const int group = blockIdx.y;
@@ -126,19 +128,11 @@ cudaError_t launch_lse_merge(int groups, int parts_per_group, int64_t rows, int 
                              const float* lse_in, void* o_out, bool out_bf16, float* lse_out, cudaStream_t st) {
   if (rows <= 0 || groups <= 0) return cudaSuccess;
   const int warps = 8;
-  dim3 grid((unsigned)((rows + warps - 1) / warps), (unsigned)groups);
-  if (d == 128) {
-    if (out_bf16)
-      lse_merge_kernel<128, true><<<grid, 32 * warps, 0, st>>>(parts_per_group, rows, o_in, lse_in, o_out, lse_out);
-    else
-      lse_merge_kernel<128, false><<<grid, 32 * warps, 0, st>>>(parts_per_group, rows, o_in, lse_in, o_out, lse_out);
-  } else {
-    if (out_bf16)
-      lse_merge_kernel<64, true><<<grid, 32 * warps, 0, st>>>(parts_per_group, rows, o_in, lse_in, o_out, lse_out);
-    else
-      lse_merge_kernel<64, false><<<grid, 32 * warps, 0, st>>>(parts_per_group, rows, o_in, lse_in, o_out, lse_out);
-  }
-  return cudaGetLastError();
+  const dim3 grid((unsigned)((rows + warps - 1) / warps), (unsigned)groups);
+  const long long nrows = rows;
+  auto kern = d == 128 ? (out_bf16 ? lse_merge_kernel<128, true> : lse_merge_kernel<128, false>)
+                       : (out_bf16 ? lse_merge_kernel<64, true> : lse_merge_kernel<64, false>);
+  return launch_pdl(kern, grid, 32 * warps, 0, st, parts_per_group, nrows, o_in, lse_in, o_out, lse_out);
 }
 
 }  // namespace star
