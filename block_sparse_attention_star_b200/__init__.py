@@ -12,6 +12,7 @@ Typical use::
     cache = star.PagedKVCache(shape, device="cuda")
     star.star_phase1_encode(shape, cache, q, k, v, pos_ctx, out)
     o_part, lse_part = star.alloc_partials(shape, T)
+    ws = star.workspace(shape, star.STAR_OP_PHASE2, T)
     star.star_phase2_partial(shape, cache, q_query, k_query, v_query, pos_query, T, o_part, lse_part, ws)
     star.star_lse_merge(shape.n, B * T * Hq, d, o_part, lse_part, out_query, lse_query)
 """
@@ -228,7 +229,7 @@ def star_phase1_encode_anchored(shape, cache: PagedKVCache, q, k, v, pos_ctx, an
                                              0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)))
 
 
-def star_phase2_partial(shape, cache: PagedKVCache, q, k, v, q_pos, T: int, o_part, lse_part, ws=None, stream=None):
+def star_phase2_partial(shape, cache: PagedKVCache, q, k, v, q_pos, T: int, o_part, lse_part, ws, stream=None):
     _check(lib().star_phase2_partial(ctypes.byref(shape), ctypes.byref(cache.c), _ptr(q, "q", torch.bfloat16),
                                      _ptr(k, "k", torch.bfloat16), _ptr(v, "v", torch.bfloat16),
                                      _ptr(q_pos, "q_pos", torch.int32), T, _ptr(o_part, "o_part", torch.float32),

@@ -154,12 +154,17 @@ int phase2_chunks_per_block(const star_shape* s, int T) {
   return best;
 }
 
+// Phase-2 scratch: RoPE(q) (bf16 [B][T][Hq][d]), then, when blocks are split into
+// chunks, the chunk partials (f32 O, then LSE).
+size_t phase2_q_bytes(const star_shape* s, int T) { return round_up((size_t)s->B * T * s->Hq * s->d * 2, 256); }
+
 size_t phase2_ws_bytes(const star_shape* s, int T) {
   const int cpb = phase2_chunks_per_block(s, T);
-  if (cpb == 1) return 0;
+  const size_t qb = phase2_q_bytes(s, T);
+  if (cpb == 1) return qb;
   const size_t rows = (size_t)s->B * T * s->Hq;
   const size_t parts = (size_t)s->n * cpb;
-  return round_up(parts * rows * s->d * sizeof(float), 256) + round_up(parts * rows * sizeof(float), 256);
+  return qb + round_up(parts * rows * s->d * sizeof(float), 256) + round_up(parts * rows * sizeof(float), 256);
 }
 
 int anchor_of(const star_shape* s) { return s->anchor ? s->anchor : s->b; }
@@ -324,13 +329,11 @@ int star_phase1_encode_anchored(const star_shape* shape, const star_cache* cache
   a.b = shape->b;
   a.n = shape->n;
   a.q = out;  // RoPE(q) is staged in the output buffer: each work item reads its Q tile, then writes O there
-  a.q_pos = pos_ctx;
   a.Ntok = shape->L;
   a.cache = cv;
   a.out_bf16 = out;
   a.chunks_per_block = 1;
   a.scale_log2 = scale_log2(shape);
-  a.rope = rt;
   const char* why = nullptr;
   trace_begin(st);
   e = star::launch_rope_q(q, pos_ctx, shape->B, shape->L, shape->Hq, shape->d, out, rt, st);
@@ -353,10 +356,8 @@ int star_phase2_partial(const star_shape* shape, const star_cache* cache, const 
   if ((k == nullptr) != (v == nullptr)) return fail(STAR_ERR_INVALID_ARG, "k and v must both be given or both be NULL");
   if (T <= 0 || T > shape->T_max) return fail(STAR_ERR_INVALID_ARG, "T (%d) must be in [1, T_max=%d]", T, shape->T_max);
   const size_t need = phase2_ws_bytes(shape, T);
-  if (need > 0) {
-    STAR_REQUIRE_PTR(ws, "ws");
-    if (ws_bytes < need) return fail(STAR_ERR_CAPACITY, "workspace %zu bytes < %zu needed", ws_bytes, need);
-  }
+  STAR_REQUIRE_PTR(ws, "ws");
+  if (ws_bytes < need) return fail(STAR_ERR_CAPACITY, "workspace %zu bytes < %zu needed", ws_bytes, need);
   cudaStream_t st = (cudaStream_t)stream;
   const star::CacheView cv = view(shape, cache);
   const star::RopeTable rt = rope_table(shape);
@@ -370,11 +371,13 @@ int star_phase2_partial(const star_shape* shape, const star_cache* cache, const 
   const int cpb = phase2_chunks_per_block(shape, T);
   const size_t rows = (size_t)shape->B * T * shape->Hq;
   const size_t parts = (size_t)shape->n * cpb;
+  void* q_rot = ws;
+  char* chunk_ws = reinterpret_cast<char*>(ws) + phase2_q_bytes(shape, T);
   float* o_dst = o_part;
   float* l_dst = lse_part;
   if (cpb > 1) {
-    o_dst = reinterpret_cast<float*>(ws);
-    l_dst = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + round_up(parts * rows * shape->d * sizeof(float), 256));
+    o_dst = reinterpret_cast<float*>(chunk_ws);
+    l_dst = reinterpret_cast<float*>(chunk_ws + round_up(parts * rows * shape->d * sizeof(float), 256));
   }
   star::AttnLaunch a;
   memset(&a, 0, sizeof(a));
@@ -387,18 +390,17 @@ int star_phase2_partial(const star_shape* shape, const star_cache* cache, const 
   a.L = shape->L;
   a.b = shape->b;
   a.n = shape->n;
-  a.q = q;
-  a.q_pos = q_pos;
+  a.q = q_rot;
   a.Ntok = T;
   a.cache = cv;
   a.out_f32 = o_dst;
   a.lse_f32 = l_dst;
   a.chunks_per_block = cpb;
   a.scale_log2 = scale_log2(shape);
-  a.rope = rt;
   const char* why = nullptr;
   trace_begin(st);
-  cudaError_t e = star::launch_attention(a, st, &why);
+  cudaError_t e = star::launch_rope_q(q, q_pos, shape->B, T, shape->Hq, shape->d, q_rot, rt, st);
+  if (e == cudaSuccess) e = star::launch_attention(a, st, &why);
   trace_end(st);
   if (e != cudaSuccess) return why ? fail(STAR_ERR_CUDA, "%s", why) : cuda_fail(e, "phase2 attention launch");
   if (cpb > 1) {

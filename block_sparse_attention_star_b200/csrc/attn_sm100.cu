@@ -34,7 +34,8 @@
 // Softmax uses the online (running max m, running sum l) formulation of the
 // FlashAttention section of the long-context attention review, in base 2 with a
 // lazily updated max: O and l are rescaled only when the tile max exceeds the
-// running max by more than 8 (so P <= 256 always fits bf16 and f32 sums).
+// running max by more than 16 (so P <= 2^16: bf16 and the f32 sums hold it with
+// the same relative precision as P <= 1, and far from overflow).
 #include "common.cuh"
 #include "internal.h"
 
@@ -50,7 +51,7 @@ constexpr int kThreads = 384;
 constexpr int kRows = 128;        // rows per Q tile (UMMA M)
 constexpr int kKeys = 128;        // keys per K/V tile (UMMA N of QK^T, K of PV)
 constexpr uint32_t kTmemCols = 512;
-constexpr float kRescaleThreshold = 8.0f;
+constexpr float kRescaleThreshold = 16.0f;
 // Per-warpgroup register budgets (setmaxnreg), chosen so neither role spills;
 // 128 x ctl + 256 x softmax must stay within the 384 x 168 registers of the launch.
 template <int D>
@@ -61,8 +62,7 @@ struct RegSplit {
 };
 
 struct Params {
-  const bf16* q;
-  const int32_t* q_pos;
+  const bf16* q;  // rotated queries (RoPE applied by the pre-pass)
   bf16* out_bf16;
   float* out_f32;
   float* lse_f32;
@@ -76,7 +76,6 @@ struct Params {
   int anchor, anchor_k_on;
   SeqShift sh;  // per-sequence context lengths L + delta[bi] (sh.on = 0: every sequence has L)
   float scale_log2;
-  double inv_freq[kMaxHalfDim];
 };
 
 struct Item {
@@ -158,9 +157,8 @@ __device__ __forceinline__ int tile_key0(const Item& it, int j) {
 struct RowInfo {
   bool valid;
   int head;       // query head
-  int tok;        // index into q / q_pos / outputs
+  int tok;        // index into q / outputs
   int cache_idx;  // cache index used by the causal rule
-  int pos;        // RoPE position
 };
 
 template <int MODE>
@@ -181,44 +179,24 @@ __device__ __forceinline__ RowInfo row_info(const Params& p, const Item& it, int
     r.tok = r.valid ? t : 0;
     r.cache_idx = r.valid ? ctx_len(p, it.bi) + t : INT_MAX;
   }
-  r.pos = r.valid ? p.q_pos[(size_t)it.bi * p.Ntok + r.tok] : 0;
   if (!r.valid) r.cache_idx = INT_MAX;
   return r;
 }
 
-// One thread writes its Q row, rotated and rounded to bf16, into the K-major
+// One thread copies its Q row (already rotated, bf16) into the K-major
 // 128-byte-swizzled tile: element (row, col) lives in the 64-column atom col/64
-// at byte row*128 + 16*((col%64/8) ^ (row%8)) + 2*(col%8).
+// at byte row*128 + 16*((col%64/8) ^ (row%8)) + 2*(col%8).  Rows past the
+// queries are zeros.
 template <int D>
 __device__ __forceinline__ void load_q_row(const Params& p, const Item& it, const RowInfo& r, uint8_t* sQ, int row) {
-  constexpr int H2 = D / 2;
   const bf16* src = p.q + (((size_t)it.bi * p.Ntok + r.tok) * p.Hq + r.head) * D;
+  uint4 v[D / 8];
 #pragma unroll
-  for (int c = 0; c < D / 16; ++c) {
-    uint4 a = make_uint4(0, 0, 0, 0), bq = make_uint4(0, 0, 0, 0);
-    if (r.valid) {
-      a = __ldg(reinterpret_cast<const uint4*>(src + 8 * c));
-      bq = __ldg(reinterpret_cast<const uint4*>(src + H2 + 8 * c));
-    }
-    const uint32_t* aw = reinterpret_cast<const uint32_t*>(&a);
-    const uint32_t* bw = reinterpret_cast<const uint32_t*>(&bq);
-    uint32_t lo[4], hi[4];
+  for (int c = 0; c < D / 8; ++c) v[c] = r.valid ? __ldg(reinterpret_cast<const uint4*>(src) + c) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      double cs[2], sn[2];
-      rope_sincos(r.pos, p.inv_freq[8 * c + 2 * e], cs[0], sn[0]);
-      rope_sincos(r.pos, p.inv_freq[8 * c + 2 * e + 1], cs[1], sn[1]);
-      rope_rotate2(aw[e], bw[e], cs, sn, lo[e], hi[e]);
-    }
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int col = half * H2 + 8 * c;
-      const int atom = col / 64;
-      const int chunk = (col % 64) / 8;
-      uint8_t* dst = sQ + atom * (kRows * 128) + row * 128 + ((chunk ^ (row & 7)) * 16);
-      const uint32_t* w = half ? hi : lo;
-      *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
+  for (int c = 0; c < D / 8; ++c) {
+    const int atom = c / 8, chunk = c % 8;
+    *reinterpret_cast<uint4*>(sQ + atom * (kRows * 128) + row * 128 + ((chunk ^ (row & 7)) * 16)) = v[c];
   }
 }
 
@@ -784,7 +762,6 @@ cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t st, const char** 
   Params p;
   memset(&p, 0, sizeof(p));
   p.q = reinterpret_cast<const bf16*>(a.q);
-  p.q_pos = a.q_pos;
   p.out_bf16 = reinterpret_cast<bf16*>(a.out_bf16);
   p.out_f32 = a.out_f32;
   p.lse_f32 = a.lse_f32;
@@ -801,7 +778,6 @@ cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t st, const char** 
   p.n = a.n;
   p.Ntok = a.Ntok;
   p.scale_log2 = a.scale_log2;
-  for (int j = 0; j < a.d / 2; ++j) p.inv_freq[j] = a.rope.inv_freq[j];
   if (a.mode == 0) {
     p.num_items = a.B * a.Hkv * a.n * (a.b / kRows) * (p.G / 2);
   } else {

@@ -89,7 +89,8 @@ struct DecSmem {
   static constexpr int kPad = kP + 2 * 2048;          // read by the N = 16 view of the last P atom
   static constexpr int kXch = kPad + 1024;            // f32 [2][4 warps][8 heads]: warp maxima
   static constexpr int kRed = kXch + 2 * 4 * 8 * 4;   // f32 [4 warps][8 heads][2]: sums
-  static constexpr int kBar = kRed + 4 * 8 * 2 * 4;
+  static constexpr int kTab = kRed + 4 * 8 * 2 * 4;   // f64 (cos, sin) [kMaxItems][D/2]: RoPE of the token
+  static constexpr int kBar = kTab + kMaxItems * (D / 2) * 16;
   static constexpr int kNumBars = 4 * kStages + 6 * 2 + 2;
   static constexpr int kSlot = kBar + kNumBars * 8;
   static constexpr int kBytes = kSlot + 16 + 1024;    // + alignment slack
@@ -244,9 +245,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   griddep_launch_dependents();
   __syncthreads();
 
+  // The token's rotation angles, once per run of items of the same sequence (the
+  // append and the G query heads of every such item use the same D/2 angles).
+  double2* tab = reinterpret_cast<double2*>(smem + S::kTab);
+  {
+    int prev_bi = -1;
+    for (int ii = 0; ii < n_my; ++ii) {
+      const int bi = dec_item(p, first + ii * gridDim.x).bi;
+      if (bi == prev_bi) continue;
+      prev_bi = bi;
+      const int tpos = p.pos[bi];
+      for (int j = threadIdx.x; j < D / 2; j += kThreads) {
+        double c, sn;
+        rope_sincos(tpos, p.inv_freq[j], c, sn);
+        tab[ii * (D / 2) + j] = make_double2(c, sn);
+      }
+    }
+  }
+  __syncthreads();
+
+  int tab_item = 0, tab_bi = -1;
   for (int ii = 0; ii < n_my; ++ii) {
     const DecItem it = dec_item(p, first + ii * gridDim.x);
-    const int tpos = p.pos[it.bi];
+    if (it.bi != tab_bi) {
+      tab_bi = it.bi;
+      tab_item = ii;
+    }
+    const double2* ang = tab + tab_item * (D / 2);
     // Append the new token (head g) when this item holds the cache's last key.
     if (it.last) {
       const int slot_abs = it.n_keys - 1;
@@ -260,9 +285,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           // pairs (j, j + 1) of the first half with the same pairs of the second half, j = 2e
           const uint32_t a = *reinterpret_cast<const uint32_t*>(p.k_new + src + 2 * e);
           const uint32_t b = *reinterpret_cast<const uint32_t*>(p.k_new + src + D / 2 + 2 * e);
-          double cs[2], sn[2];
-          rope_sincos(tpos, p.inv_freq[2 * e], cs[0], sn[0]);
-          rope_sincos(tpos, p.inv_freq[2 * e + 1], cs[1], sn[1]);
+          const double2 a0 = ang[2 * e], a1 = ang[2 * e + 1];
+          const double cs[2] = {a0.x, a1.x}, sn[2] = {a0.y, a1.y};
           uint32_t lo, hi;
           rope_rotate2(a, b, cs, sn, lo, hi);
           *reinterpret_cast<uint32_t*>(p.kpool + dst + 2 * e) = lo;
@@ -281,8 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int h = e / (D / 2), j = e % (D / 2);
       const bf16* qr = p.q + ((size_t)it.bi * p.Hq + it.g * G + h) * D;
       const double x1 = __bfloat162float(qr[j]), x2 = __bfloat162float(qr[j + D / 2]);
-      double cs, sn;
-      rope_sincos(tpos, p.inv_freq[j], cs, sn);
+      const double cs = ang[j].x, sn = ang[j].y;
       const int d1 = j, d2 = j + D / 2;
       *reinterpret_cast<bf16*>(qs + (d1 / 64) * 1024 + sw128(h, d1 % 64)) = __double2bfloat16(x1 * cs - x2 * sn);
       *reinterpret_cast<bf16*>(qs + (d2 / 64) * 1024 + sw128(h, d2 % 64)) = __double2bfloat16(x2 * cs + x1 * sn);

@@ -86,8 +86,7 @@ cudaError_t launch_lse_merge(int groups, int parts_per_group, int64_t rows, int 
 struct AttnLaunch {
   int mode;               // 0: Phase-1 context attention, 1: Phase-2 query partials
   int B, Hq, Hkv, d, L, b, n;
-  const void* q;          // [B][Ntok][Hq][d] bf16: mode 0 already rotated (staged by TMA), mode 1 pre-RoPE
-  const int32_t* q_pos;   // [B][Ntok]
+  const void* q;          // [B][Ntok][Hq][d] bf16, already rotated (mode 0: staged by TMA, mode 1: by threads)
   int Ntok;
   CacheView cache;
   void* out_bf16;         // mode 0: [B][L][Hq][d]
@@ -98,7 +97,6 @@ struct AttnLaunch {
   SeqShift shift;         // per-sequence context lengths L + delta[s] (on = 0: all L)
   const void* anchor_k;   // mode 0: NULL (anchor keys are block 1's cached keys) or bf16 [B][n-1][Hkv][a][d]
   float scale_log2;
-  RopeTable rope;
 };
 int attn_num_parts(const AttnLaunch& a);  // mode 1: n * chunks_per_block
 cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t st, const char** why);

@@ -83,18 +83,25 @@ __global__ void __launch_bounds__(256) rope_append_kernel(const bf16* __restrict
 
 // RoPE of the query heads of ntok tokens per sequence: out[b][t][h] = rotation of
 // q[b][t][h] at pos[b][t] (float64 rotation, one bf16 rounding, as the keys).  One
-// thread per (sequence, token, 8-pair chunk): the 8 angles are computed once and
-// applied to that chunk of every query head.  out may be q itself: each element is
-// read and then written by the same thread.
+// thread per (head group, sequence, token, 8-pair chunk): the 8 angles are computed
+// once and applied to that chunk of the group's hpt heads, four heads' loads in
+// flight at a time.  Long inputs use one group of all H heads (each angle computed
+// once); a few tokens split the heads over more threads, so that the kernel is not
+// one serial chain of loads per thread.  out may be q itself: each element is read
+// and then written by the same thread.
 template <int D>
 __global__ void __launch_bounds__(256) rope_q_kernel(const bf16* q, const int32_t* __restrict__ pos, int B, int ntok,
-                                                     int H, bf16* out, const __grid_constant__ RopeParams rp) {
+                                                     int H, int hpt, bf16* out, const __grid_constant__ RopeParams rp) {
   constexpr int CH = D / 16;
-  const long long total = (long long)B * ntok * CH;
+  const int HG = (H + hpt - 1) / hpt;
+  const long long rows = (long long)B * ntok;
+  const long long total = rows * CH * HG;
   for (long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x; gid < total;
        gid += (long long)gridDim.x * blockDim.x) {
     const int c = (int)(gid % CH);
-    const long long r = gid / CH;  // bi * ntok + t
+    const long long rest = gid / CH;
+    const long long r = rest % rows;  // bi * ntok + t
+    const int hg = (int)(rest / rows);
     const int p_t = pos[r];
     double cs[4][2], sn[4][2];
 #pragma unroll
@@ -102,17 +109,30 @@ __global__ void __launch_bounds__(256) rope_q_kernel(const bf16* q, const int32_
       rope_sincos(p_t, rp.inv_freq[8 * c + 2 * e], cs[e][0], sn[e][0]);
       rope_sincos(p_t, rp.inv_freq[8 * c + 2 * e + 1], cs[e][1], sn[e][1]);
     }
-    for (int h = 0; h < H; ++h) {
-      const size_t off = ((size_t)r * H + h) * D;
-      const uint4 a = *reinterpret_cast<const uint4*>(q + off + 8 * c);
-      const uint4 bq = *reinterpret_cast<const uint4*>(q + off + D / 2 + 8 * c);
-      const uint32_t* aw = reinterpret_cast<const uint32_t*>(&a);
-      const uint32_t* bw = reinterpret_cast<const uint32_t*>(&bq);
-      uint32_t lo[4], hi[4];
+    const int h1 = min(H, (hg + 1) * hpt);
+    for (int h0 = hg * hpt; h0 < h1; h0 += 4) {
+      uint4 a[4], bq[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) rope_rotate2(aw[e], bw[e], cs[e], sn[e], lo[e], hi[e]);
-      *reinterpret_cast<uint4*>(out + off + 8 * c) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-      *reinterpret_cast<uint4*>(out + off + D / 2 + 8 * c) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      for (int u = 0; u < 4; ++u) {
+        if (h0 + u < h1) {
+          const size_t off = ((size_t)r * H + h0 + u) * D;
+          a[u] = *reinterpret_cast<const uint4*>(q + off + 8 * c);
+          bq[u] = *reinterpret_cast<const uint4*>(q + off + D / 2 + 8 * c);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (h0 + u < h1) {
+          const size_t off = ((size_t)r * H + h0 + u) * D;
+          const uint32_t* aw = reinterpret_cast<const uint32_t*>(&a[u]);
+          const uint32_t* bw = reinterpret_cast<const uint32_t*>(&bq[u]);
+          uint32_t lo[4], hi[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) rope_rotate2(aw[e], bw[e], cs[e], sn[e], lo[e], hi[e]);
+          *reinterpret_cast<uint4*>(out + off + 8 * c) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          *reinterpret_cast<uint4*>(out + off + D / 2 + 8 * c) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        }
+      }
     }
   }
 }
@@ -255,13 +275,16 @@ cudaError_t launch_rope_q(const void* q, const int32_t* pos, int B, int ntok, in
   if (ntok <= 0 || B <= 0) return cudaSuccess;
   RopeParams rp;
   for (int j = 0; j < d / 2; ++j) rp.inv_freq[j] = rt.inv_freq[j];
-  const long long work = (long long)B * ntok * (d / 16);
-  const int grid = grid_for(work, 256);
+  // Head groups: enough threads to fill the GPU (148 SMs x 1024), at most one head each.
+  const long long base = (long long)B * ntok * (d / 16);
+  const long long groups = std::min<long long>(H, std::max<long long>(1, 148LL * 1024 / base));
+  const int hpt = (int)((H + groups - 1) / groups);
+  const int grid = grid_for(base * ((H + hpt - 1) / hpt), 256);
   if (d == 128)
-    rope_q_kernel<128><<<grid, 256, 0, st>>>(reinterpret_cast<const bf16*>(q), pos, B, ntok, H,
+    rope_q_kernel<128><<<grid, 256, 0, st>>>(reinterpret_cast<const bf16*>(q), pos, B, ntok, H, hpt,
                                              reinterpret_cast<bf16*>(out), rp);
   else
-    rope_q_kernel<64><<<grid, 256, 0, st>>>(reinterpret_cast<const bf16*>(q), pos, B, ntok, H,
+    rope_q_kernel<64><<<grid, 256, 0, st>>>(reinterpret_cast<const bf16*>(q), pos, B, ntok, H, hpt,
                                             reinterpret_cast<bf16*>(out), rp);
   return cudaGetLastError();
 }

@@ -118,7 +118,10 @@ int star_page_table_fill(const star_shape* shape, int32_t* page_table_host, int3
 /* Bytes of scratch the given operation needs (op = STAR_OP_*; for STAR_OP_PHASE2
  * T is the number of query tokens of the call, ignored otherwise).
  * STAR_OP_PHASE1: 0.  STAR_OP_PHASE1_ANCHOR: star_phase1_encode_anchored with anchor
- * position ids, B*(n-1)*Hkv*a*d*2 bytes (the anchor's keys roped at those ids). */
+ * position ids, B*(n-1)*Hkv*a*d*2 bytes (the anchor's keys roped at those ids).
+ * STAR_OP_PHASE2: RoPE(q) (B*T*Hq*d*2 bytes, rounded up to 256), plus the f32 partials
+ * of the chunks when blocks are split to fill the GPU.  STAR_OP_DECODE: the chunk
+ * partials of one step. */
 int star_workspace_size(const star_shape* shape, int op, int32_t T, size_t* bytes_out);
 
 /* Integer structure of c' ("被增广的上下文"), for checking only.
@@ -176,6 +179,7 @@ int star_phase1_encode_anchored(const star_shape* shape, const star_cache* cache
  * and, in block n, its b context keys plus tail keys L..L+t.
  * o_part: f32 [n][B][T][Hq][d], normalised local outputs A_i;
  * lse_part: f32 [n][B][T][Hq], log s_i.  T <= T_max.
+ * ws: at least star_workspace_size(STAR_OP_PHASE2, T) bytes (never NULL).
  * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, ALIGNMENT, CAPACITY, CUDA. */
 int star_phase2_partial(const star_shape* shape, const star_cache* cache, const void* q, const void* k,
                         const void* v, const int32_t* q_pos, int32_t T, float* o_part, float* lse_part, void* ws,
