@@ -26,16 +26,16 @@
 // HBM rate instead of being bound by instruction issue, as a CUDA-core dot-product
 // formulation of the same step is (about 80 instructions per key and head group).
 //
-// Before any load, the CTA owning the last chunk of a (sequence, KV head) appends
-// the new token: RoPE(k) (float64 rotation, one bf16 rounding, like
-// star_kv_append) and v go to cache slot n_keys - 1, made visible to its own TMA
-// loads by a proxy fence.
+// The CTA owning the last chunk of a (sequence, KV head) appends the new token:
+// RoPE(k) (float64 rotation, one bf16 rounding, like star_kv_append) and v go to
+// cache slot n_keys - 1, made visible to its own TMA loads by a proxy fence and an
+// mbarrier that the producer waits on before the tile holding that slot.
 //
 // CTA (256 threads, one per SM):
 //   warp 0     TMA producer (K and V rings, no multicast)
 //   warp 1     TMEM allocation and MMA issuer
-//   warps 2-3  prologue only (appends, q)
-//   warps 4-7  softmax and O accumulation: thread = TMEM lane 32 (w - 4) + lane
+//   warps 2-7  prologue (append, q) while warp 0 already streams K and V
+//   warps 4-7  then softmax and O accumulation: thread = TMEM lane 32 (w - 4) + lane
 #include "common.cuh"
 #include "internal.h"
 
@@ -48,6 +48,8 @@ constexpr int kThreads = 256;
 constexpr int kTileKeys = 128;           // UMMA M of S^T, K of O^T
 constexpr int kStages = 3;               // K/V ring depth
 constexpr int kMaxItems = 8;             // items per CTA per launch (q of each stays in shared memory)
+constexpr int kProWarps = 6;             // warps 2-7 run the prologue (append, q)
+constexpr int kProThreads = 32 * kProWarps;
 constexpr uint32_t kTmemCols = 64;       // S^T: [0,16) [16,32); O^T: [32,48) [48,64)
 constexpr uint32_t kIdescQK = umma_idesc_bf16(128, 16, 0, 0);
 constexpr uint32_t kIdescPV = umma_idesc_bf16(128, 16, 1, 0);
@@ -90,8 +92,9 @@ struct DecSmem {
   static constexpr int kXch = kPad + 1024;            // f32 [2][4 warps][8 heads]: warp maxima
   static constexpr int kRed = kXch + 2 * 4 * 8 * 4;   // f32 [4 warps][8 heads][2]: sums
   static constexpr int kTab = kRed + 4 * 8 * 2 * 4;   // f64 (cos, sin) [kMaxItems][D/2]: RoPE of the token
-  static constexpr int kBar = kTab + kMaxItems * (D / 2) * 16;
-  static constexpr int kNumBars = 4 * kStages + 6 * 2 + 2;
+  static constexpr int kTabOf = kTab + kMaxItems * (D / 2) * 16;  // int [kMaxItems]: table used by each item
+  static constexpr int kBar = kTabOf + kMaxItems * 4;
+  static constexpr int kNumBars = 4 * kStages + 6 * 2 + 3;
   static constexpr int kSlot = kBar + kNumBars * 8;
   static constexpr int kBytes = kSlot + 16 + 1024;    // + alignment slack
   static_assert(kBytes <= 227 * 1024, "decode shared memory");
@@ -201,6 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* x_bar = s_full + 10;
   uint64_t* red_bar = s_full + 12;
   uint64_t* drain = s_full + 13;
+  uint64_t* pro_done = s_full + 14;  // warps 2-7 have appended the token and staged q
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kSlot);
   float* xch = reinterpret_cast<float*>(smem + S::kXch);
   float* red = reinterpret_cast<float*>(smem + S::kRed);
@@ -226,6 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(red_bar, 4);
     mbar_init(drain, 1);
+    mbar_init(pro_done, kProWarps);
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -239,83 +244,104 @@ __global__ void __launch_bounds__(kThreads, 1)
   // q and P operands: the padding rows (heads G..15) are zeros.
   for (int i = threadIdx.x; i < (S::kXch - S::kQ) / 16; i += kThreads)
     reinterpret_cast<uint4*>(smem + S::kQ)[i] = make_uint4(0u, 0u, 0u, 0u);
+  fence_proxy_async_smem();
   // Everything above touches only this CTA's on-chip state, so it overlaps the
   // previous kernel's tail; global memory is read and written only after it ends.
   griddep_wait();
   griddep_launch_dependents();
-  __syncthreads();
-
-  // The token's rotation angles, once per run of items of the same sequence (the
-  // append and the G query heads of every such item use the same D/2 angles).
-  double2* tab = reinterpret_cast<double2*>(smem + S::kTab);
-  {
-    int prev_bi = -1;
-    for (int ii = 0; ii < n_my; ++ii) {
-      const int bi = dec_item(p, first + ii * gridDim.x).bi;
-      if (bi == prev_bi) continue;
-      prev_bi = bi;
-      const int tpos = p.pos[bi];
-      for (int j = threadIdx.x; j < D / 2; j += kThreads) {
-        double c, sn;
-        rope_sincos(tpos, p.inv_freq[j], c, sn);
-        tab[ii * (D / 2) + j] = make_double2(c, sn);
-      }
-    }
-  }
-  __syncthreads();
-
-  int tab_item = 0, tab_bi = -1;
-  for (int ii = 0; ii < n_my; ++ii) {
-    const DecItem it = dec_item(p, first + ii * gridDim.x);
-    if (it.bi != tab_bi) {
-      tab_bi = it.bi;
-      tab_item = ii;
-    }
-    const double2* ang = tab + tab_item * (D / 2);
-    // Append the new token (head g) when this item holds the cache's last key.
-    if (it.last) {
-      const int slot_abs = it.n_keys - 1;
-      const int page = p.page_table[(size_t)it.bi * p.max_pages + slot_abs / p.P];
-      if (page < 0 || page >= p.num_pages) {
-        if (threadIdx.x == 0) record_error(kDevBadPage);
-      } else {
-        const size_t dst = (((size_t)page * p.Hkv + it.g) * p.P + (slot_abs % p.P)) * D;
-        const size_t src = ((size_t)it.bi * p.Hkv + it.g) * D;
-        for (int e = threadIdx.x; e < D / 4; e += kThreads) {
-          // pairs (j, j + 1) of the first half with the same pairs of the second half, j = 2e
-          const uint32_t a = *reinterpret_cast<const uint32_t*>(p.k_new + src + 2 * e);
-          const uint32_t b = *reinterpret_cast<const uint32_t*>(p.k_new + src + D / 2 + 2 * e);
-          const double2 a0 = ang[2 * e], a1 = ang[2 * e + 1];
-          const double cs[2] = {a0.x, a1.x}, sn[2] = {a0.y, a1.y};
-          uint32_t lo, hi;
-          rope_rotate2(a, b, cs, sn, lo, hi);
-          *reinterpret_cast<uint32_t*>(p.kpool + dst + 2 * e) = lo;
-          *reinterpret_cast<uint32_t*>(p.kpool + dst + D / 2 + 2 * e) = hi;
-        }
-        for (int e = threadIdx.x; e < D / 2; e += kThreads)
-          *reinterpret_cast<uint32_t*>(p.vpool + dst + 2 * e) =
-              *reinterpret_cast<const uint32_t*>(p.v_new + src + 2 * e);
-        fence_proxy_async_global();
-      }
-    }
-    // q of the G heads: RoPE at the token's position (float64 rotation, one bf16
-    // rounding, as the cache keys), as the K-major B operand [head][d].
-    uint8_t* qs = smem + S::kQ + ii * S::kQItem;
-    for (int e = threadIdx.x; e < G * (D / 2); e += kThreads) {
-      const int h = e / (D / 2), j = e % (D / 2);
-      const bf16* qr = p.q + ((size_t)it.bi * p.Hq + it.g * G + h) * D;
-      const double x1 = __bfloat162float(qr[j]), x2 = __bfloat162float(qr[j + D / 2]);
-      const double cs = ang[j].x, sn = ang[j].y;
-      const int d1 = j, d2 = j + D / 2;
-      *reinterpret_cast<bf16*>(qs + (d1 / 64) * 1024 + sw128(h, d1 % 64)) = __double2bfloat16(x1 * cs - x2 * sn);
-      *reinterpret_cast<bf16*>(qs + (d2 / 64) * 1024 + sw128(h, d2 % 64)) = __double2bfloat16(x2 * cs + x1 * sn);
-    }
-  }
-  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
+
+  // Warps 2-7 append the token and stage q (below) while the producer already
+  // streams K and V; the producer waits for the append only before the tile that
+  // holds the new slot, and the MMA warp waits for q before its first product.
+  if (warp >= 2) {
+    const int pt = threadIdx.x - 64;
+    // The token's rotation angles, once per run of items of the same sequence (the
+    // append and the G query heads of every such item use the same D/2 angles);
+    // tab_of[ii] is the item whose table item ii uses.
+    double2* tab = reinterpret_cast<double2*>(smem + S::kTab);
+    int* tab_of = reinterpret_cast<int*>(smem + S::kTabOf);
+    {
+      int prev_bi = -1, cur = 0;
+      for (int ii = 0; ii < n_my; ++ii) {
+        const int bi = dec_item(p, first + ii * gridDim.x).bi;
+        if (bi != prev_bi) {
+          prev_bi = bi;
+          cur = ii;
+          const int tpos = p.pos[bi];
+          for (int j = pt; j < D / 2; j += kProThreads) {
+            double c, sn;
+            rope_sincos(tpos, p.inv_freq[j], c, sn);
+            tab[ii * (D / 2) + j] = make_double2(c, sn);
+          }
+        }
+        if (pt == 0) tab_of[ii] = cur;
+      }
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kProThreads) : "memory");
+
+    // Append the new token (head g) for each item that holds its sequence's last key.
+    for (int ii = 0; ii < n_my; ++ii) {
+      const DecItem it = dec_item(p, first + ii * gridDim.x);
+      if (!it.last) continue;
+      const double2* ang = tab + tab_of[ii] * (D / 2);
+      const int slot_abs = it.n_keys - 1;
+      const int page = p.page_table[(size_t)it.bi * p.max_pages + slot_abs / p.P];
+      if (page < 0 || page >= p.num_pages) {
+        if (pt == 0) record_error(kDevBadPage);
+        continue;
+      }
+      const size_t dst = (((size_t)page * p.Hkv + it.g) * p.P + (slot_abs % p.P)) * D;
+      const size_t src = ((size_t)it.bi * p.Hkv + it.g) * D;
+      for (int e = pt; e < D / 4; e += kProThreads) {
+        // pairs (j, j + 1) of the first half with the same pairs of the second half, j = 2e
+        const uint32_t a = *reinterpret_cast<const uint32_t*>(p.k_new + src + 2 * e);
+        const uint32_t b = *reinterpret_cast<const uint32_t*>(p.k_new + src + D / 2 + 2 * e);
+        const double2 a0 = ang[2 * e], a1 = ang[2 * e + 1];
+        const double cs[2] = {a0.x, a1.x}, sn[2] = {a0.y, a1.y};
+        uint32_t lo, hi;
+        rope_rotate2(a, b, cs, sn, lo, hi);
+        *reinterpret_cast<uint32_t*>(p.kpool + dst + 2 * e) = lo;
+        *reinterpret_cast<uint32_t*>(p.kpool + dst + D / 2 + 2 * e) = hi;
+      }
+      for (int e = pt; e < D / 2; e += kProThreads)
+        *reinterpret_cast<uint32_t*>(p.vpool + dst + 2 * e) = *reinterpret_cast<const uint32_t*>(p.v_new + src + 2 * e);
+    }
+
+    // q of the G heads of every item: RoPE at the token's position (float64 rotation,
+    // one bf16 rounding, as the cache keys), as the K-major B operand [head][d].  A
+    // unit is 8 rotation pairs of one head: two 16-byte loads, two 16-byte stores.
+    constexpr int kUnits = G * (D / 16);
+    for (int u = pt; u < n_my * kUnits; u += kProThreads) {
+      const int ii = u / kUnits, h = (u % kUnits) / (D / 16), c = u % (D / 16);
+      const DecItem it = dec_item(p, first + ii * gridDim.x);
+      const bf16* qr = p.q + ((size_t)it.bi * p.Hq + it.g * G + h) * D;
+      const uint4 a = __ldg(reinterpret_cast<const uint4*>(qr + 8 * c));
+      const uint4 b = __ldg(reinterpret_cast<const uint4*>(qr + D / 2 + 8 * c));
+      const double2* ang = tab + tab_of[ii] * (D / 2) + 8 * c;
+      const uint32_t* aw = reinterpret_cast<const uint32_t*>(&a);
+      const uint32_t* bw = reinterpret_cast<const uint32_t*>(&b);
+      uint32_t lo[4], hi[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const double2 a0 = ang[2 * e], a1 = ang[2 * e + 1];
+        const double cs[2] = {a0.x, a1.x}, sn[2] = {a0.y, a1.y};
+        rope_rotate2(aw[e], bw[e], cs, sn, lo[e], hi[e]);
+      }
+      uint8_t* qs = smem + S::kQ + ii * S::kQItem;
+      const int d1 = 8 * c, d2 = D / 2 + 8 * c;
+      *reinterpret_cast<uint4*>(qs + (d1 / 64) * 1024 + sw128(h, d1 % 64)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      *reinterpret_cast<uint4*>(qs + (d2 / 64) * 1024 + sw128(h, d2 % 64)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    }
+    // The appended K/V (global) and q (shared) are read next by the async proxy (TMA, MMA).
+    fence_proxy_async_global();
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(pro_done);
+  }
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
@@ -326,6 +352,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const DecItem it = dec_item(p, first + ii * gridDim.x);
         for (int t = 0; t < it.ntiles && ok; ++t, ++kc) {
           const int k0 = it.k_begin + t * kTileKeys;
+          // The tile holding the new token's slot is loaded after the append.
+          if (it.last && t == it.ntiles - 1 && !mbar_wait(pro_done, 0, kDevTimeoutProducer)) {
+            ok = false;
+            break;
+          }
           int page = p.page_table[(size_t)it.bi * p.max_pages + k0 / p.P];
           if (page < 0 || page >= p.num_pages) {
             record_error(kDevBadPage);
@@ -381,7 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       uint32_t j = 0;
-      bool ok = true;
+      bool ok = mbar_wait(pro_done, 0, kDevTimeoutMma);  // q of every item is staged
       for (int ii = 0; ii < n_my && ok; ++ii) {
         const DecItem it = dec_item(p, first + ii * gridDim.x);
         const uint32_t qa = sQ + ii * S::kQItem;
