@@ -34,8 +34,9 @@
 // Softmax uses the online (running max m, running sum l) formulation of the
 // FlashAttention section of the long-context attention review, in base 2 with a
 // lazily updated max: O and l are rescaled only when the tile max exceeds the
-// running max by more than 16 (so P <= 2^16: bf16 and the f32 sums hold it with
-// the same relative precision as P <= 1, and far from overflow).
+// running max by more than 32 (so P <= 2^32: bf16 and f32 hold it with the same
+// relative precision as P <= 1, and a row's f32 sums stay below 2^52 for up to
+// 2^20 keys, far from overflow).
 #include "common.cuh"
 #include "internal.h"
 
@@ -51,7 +52,7 @@ constexpr int kThreads = 384;
 constexpr int kRows = 128;        // rows per Q tile (UMMA M)
 constexpr int kKeys = 128;        // keys per K/V tile (UMMA N of QK^T, K of PV)
 constexpr uint32_t kTmemCols = 512;
-constexpr float kRescaleThreshold = 16.0f;
+constexpr float kRescaleThreshold = 32.0f;
 // Per-warpgroup register budgets (setmaxnreg), chosen so neither role spills;
 // 128 x ctl + 256 x softmax must stay within the 384 x 168 registers of the launch.
 template <int D>
