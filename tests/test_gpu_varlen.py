@@ -40,6 +40,10 @@ SMALL = {
     "tiny-ragged": dataclasses.replace(get_config("tiny"), name="tiny-ragged", seq_lens=(777,)),
     "d128-g8-var-t130": Workload("d128-g8-var-t130", B=2, Hq=16, Hkv=2, d=128, L=1024, b=256, T=130, S=2,
                                  peaky=True, seq_lens=(1024, 333)),
+    # six sequences, the shortest first and a one-token context: per-sequence item tables
+    # and chunk counts in the decode (one chunk for the first sequence, four for the third)
+    "d64-g4-var-b6": Workload("d64-g4-var-b6", B=6, Hq=8, Hkv=2, d=64, L=1024, b=256, T=9, S=2, peaky=True,
+                              seq_lens=(1, 130, 1024, 257, 640, 999)),
 }
 
 
