@@ -143,6 +143,15 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # The CUDA path
 # ---------------------------------------------------------------------------
+def workload_config(wl, world):
+    """The `config` object of the JSON line (the same for both arms)."""
+    return {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d, "L": wl.L, "b": wl.b,
+            "n": wl.n, "T": wl.T, "S": wl.S, "page_tokens": wl.page_tokens, "anchor": wl.a,
+            "anchor_ids": wl.anchor_ids, "seq_lens": list(wl.seq_lens) if wl.seq_lens else None,
+            "parallelism": f"independent sequences per GPU x{world}",
+            "l2": "inputs larger than L2 (no flush)"}
+
+
 def workload_shape(wl):
     """The C-ABI shape of a workload: sizes, anchor and per-sequence context lengths."""
     import block_sparse_attention_star_b200 as star
@@ -340,11 +349,7 @@ def run_star(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": max(3, args.warmup),
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16; 1% of context key rows x8 where the workload says peaky)",
-        "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d, "L": wl.L, "b": wl.b,
-                   "n": wl.n, "T": wl.T, "S": wl.S, "page_tokens": wl.page_tokens, "anchor": wl.a,
-                   "anchor_ids": wl.anchor_ids, "seq_lens": list(wl.seq_lens) if wl.seq_lens else None,
-                   "parallelism": f"independent sequences per GPU x{world}",
-                   "l2": "inputs larger than L2 (no flush)"},
+        "config": workload_config(wl, world),
         "phase1": {"attn_ms": p1_ms, "ctx_tok_s": wl.context_tokens() / (p1_ms * 1e-3), "tflops": tflops,
                    "frac_bf16_burst": tflops / peaks["bf16"], "frac_bf16_sustained": tflops / peaks["bf16_sustained"]},
         "phase2": {"attn_ms": p2_ms},
@@ -520,8 +525,7 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": W, "ms_per_step": 1e3 * tot_sec / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (same seeded inputs as the CUDA arm)",
-        "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d, "L": wl.L, "b": wl.b,
-                   "n": wl.n, "T": wl.T, "S": wl.S, "anchor": wl.a, "anchor_ids": wl.anchor_ids},
+        "config": workload_config(wl, world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
                          "sample": f"each step: float64 oracle Phase-1 output of {rows_per_block} context rows of one "
                                    f"block (all {wl.Hq} heads) of {wl.name}; value = rows/s"},
