@@ -99,3 +99,25 @@ def test_null_arguments_rejected_before_any_launch():
     assert rc == star.STAR_ERR_UNSUPPORTED_SHAPE
     rc = lib.star_set_trace_events(ctypes.c_void_p(16), None)
     assert rc == star.STAR_ERR_INVALID_ARG
+
+
+def test_phase2_and_decode_workspaces_are_checked_before_any_launch():
+    """Phase 2 always needs its workspace (RoPE(q) is staged there); both calls check its size."""
+    lib = star.lib()
+    sh = _shape()
+    max_pages = ctypes.c_int32()
+    assert lib.star_pages_needed(ctypes.byref(sh), ctypes.byref(max_pages)) == star.STAR_OK
+    # Never dereferenced: every call below fails its argument checks first.
+    cache = star.StarCache(k_pool=256, v_pool=256, page_table=256, max_pages=max_pages.value, num_pages=1)
+    p = ctypes.c_void_p(256)
+    T = 64
+    need = star.star_workspace_size(sh, star.STAR_OP_PHASE2, T)
+    assert need >= sh.B * T * sh.Hq * sh.d * 2
+    rc = lib.star_phase2_partial(ctypes.byref(sh), ctypes.byref(cache), p, None, None, p, T, p, p, None, 0, None)
+    assert rc == star.STAR_ERR_INVALID_ARG  # ws is NULL
+    rc = lib.star_phase2_partial(ctypes.byref(sh), ctypes.byref(cache), p, None, None, p, T, p, p, p, need - 256, None)
+    assert rc == star.STAR_ERR_CAPACITY
+    need_d = star.star_workspace_size(sh, star.STAR_OP_DECODE)
+    rc = lib.star_decode_step(ctypes.byref(sh), ctypes.byref(cache), p, p, p, p, sh.L, p, None, p, need_d - 256,
+                              None)
+    assert rc == star.STAR_ERR_CAPACITY
