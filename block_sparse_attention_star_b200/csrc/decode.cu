@@ -699,12 +699,6 @@ int decode_pick_chunk(int B, int Hkv, int G, int n_keys, int num_sms) {
   return (int)(best_ct * kTileKeys);
 }
 
-size_t decode_smem_bytes(int d, int G, int chunk) {
-  (void)G;
-  (void)chunk;
-  return d == 128 ? DecSmem<128>::kBytes : DecSmem<64>::kBytes;
-}
-
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t st) {
   DecParams p;
   p.q = reinterpret_cast<const bf16*>(a.q);

@@ -120,7 +120,6 @@ struct DecodeLaunch {
 int decode_num_chunks(int n_keys, int chunk);
 int decode_pick_chunk(int B, int Hkv, int G, int n_keys, int num_sms);
 int decode_pick_chunk_var(int B, int Hkv, const int* n_keys_of, int min_chunk, int num_sms);
-size_t decode_smem_bytes(int d, int G, int chunk);
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t st);
 
 // --- api.cu: the thread-local message read by star_last_error(); returns code ----
