@@ -93,10 +93,6 @@ class Workload:
     def ctx_len(self, bi: int) -> int:
         return self.seq_lens[bi] if self.seq_lens is not None else self.L
 
-    def kv_bytes(self, tokens: int) -> int:
-        """bf16 K plus V bytes for ``tokens`` cached tokens of every sequence."""
-        return tokens * self.Hkv * self.d * 2 * 2 * self.B
-
     def decode_bytes(self, step: int) -> int:
         """K and V bytes one decode step reads: every sequence's context, query tail, the
         tokens generated before and the new one."""
