@@ -10,6 +10,7 @@ synthetic tensors already resident in HBM when the timed region starts; the
 timed region.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl star|reference]
+    python bench.py --layers N [--config NAME]   # N layers of context encoding (star_encode_layers)
 
 Multi-GPU (torchrun): every rank runs its own independent sequence batch (the
 path partitions by sequence; no collective on the data path); time is the max
@@ -50,6 +51,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=8, help="Phase-1 rows per block in the oracle sample")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="time N layers of context encoding (star_encode_layers, random projections) instead")
     return ap.parse_args()
 
 
@@ -534,6 +537,72 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_layers(args):
+    """Context encoding through `args.layers` layers on one GPU: per layer the caller's
+    projections (random bf16 weights, cuBLAS through torch, in the layer callback) and the
+    library's Phase 1 (RoPE + KV append + anchor-augmented attention).  One step = the
+    whole stack over the workload's context; inputs resident in HBM."""
+    import block_sparse_attention_star_b200 as star
+    from synth import layer_inputs
+    wl = get_config(args.config)
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    nl, B, L, Hq, Hkv, d = args.layers, wl.B, wl.L, wl.Hq, wl.Hkv, wl.d
+    hidden = Hq * d
+    x0, ws = layer_inputs(wl.seed, nl, B, L, hidden, Hq * d, Hkv * d, device=dev)
+    shape = workload_shape(dataclasses.replace(wl, seq_lens=None))
+    caches = [star.PagedKVCache(shape, device=dev) for _ in range(nl)]
+    pos = torch.arange(L, dtype=torch.int32, device=dev).repeat(B, 1).contiguous()
+    x = x0.clone()
+    q = torch.empty((B, L, Hq, d), dtype=torch.bfloat16, device=dev)
+    k = torch.empty((B, L, Hkv, d), dtype=torch.bfloat16, device=dev)
+    v, o = torch.empty_like(k), torch.empty_like(q)
+
+    def model(layer, stage, x, q, k, v, o):
+        wq, wk, wv, wo = ws[layer]
+        xf = x.view(B * L, hidden)
+        if stage == star.STAR_LAYER_QKV:
+            torch.matmul(xf, wq, out=q.view(B * L, Hq * d))
+            torch.matmul(xf, wk, out=k.view(B * L, Hkv * d))
+            torch.matmul(xf, wv, out=v.view(B * L, Hkv * d))
+        else:
+            xf.add_(torch.matmul(o.view(B * L, Hq * d), wo))
+
+    def step(attn_ev=None):
+        x.copy_(x0)
+        if attn_ev:
+            star.star_set_trace_events(*attn_ev)
+        star.star_encode_layers(shape, caches, pos, x, q, k, v, o, model)
+        if attn_ev:
+            star.star_set_trace_events(None, None)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    K = args.steps
+    t0, t1 = _ev(), _ev()
+    t0.record()
+    for _ in range(K):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / K
+    attn = _pair()  # the last layer's Phase 1 (each layer re-records the pair), one extra untimed step
+    step(attn)
+    torch.cuda.synchronize()
+    attn_ms = attn[0].elapsed_time(attn[1])
+    status = star.star_device_status()
+    proj_flop = 2.0 * B * L * hidden * (Hq * d + 2 * Hkv * d) + 2.0 * B * L * Hq * d * hidden
+    line = {"metric": f"context encoding through {nl} layers (ctx tok/s)", "value": wl.context_tokens() / (ms * 1e-3),
+            "unit": UNIT, "n_gpus": 1, "steps": K, "warmup": max(3, args.warmup), "ms_per_step": ms,
+            "higher_is_better": True, "dtype": "bf16", "data": "synthetic (seeded N(0,1) hidden states, random weights)",
+            "config": dict(workload_config(wl, 1), layers=nl, hidden=hidden),
+            "per_layer_ms": ms / nl, "attention_ms_per_layer": attn_ms,
+            "attention_tflops": wl.phase1_flops() / (attn_ms * 1e-3) / 1e12,
+            "projection_flop_per_layer": proj_flop, "device_status": status}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -541,6 +610,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.layers > 0:
+        run_layers(args)
         return
     if world > 1:
         import datetime

@@ -36,6 +36,8 @@ STAR_ERR_ALIGNMENT = -3
 STAR_ERR_CAPACITY = -4
 STAR_ERR_CUDA = -5
 STAR_ERR_TIMEOUT = -6
+STAR_ERR_CALLBACK = -7
+STAR_LAYER_QKV, STAR_LAYER_OUT = 0, 1
 STAR_OP_PHASE1, STAR_OP_PHASE2, STAR_OP_DECODE, STAR_OP_PHASE1_ANCHOR = 1, 2, 3, 4
 
 
@@ -78,6 +80,10 @@ class StarCache(ctypes.Structure):
 
 _lib = None
 
+# int fn(int32 layer, int32 stage, void* in, void* out0, void* out1, void* out2, void* user, stream)
+LAYER_FN = ctypes.CFUNCTYPE(ctypes.c_int, ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
+                            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p)
+
 
 def lib() -> ctypes.CDLL:
     """The loaded libstar.so (raises if it has not been built)."""
@@ -103,6 +109,7 @@ def lib() -> ctypes.CDLL:
             "star_device_status": ([V, P(I32)], ctypes.c_int),
             "star_set_trace_events": ([V, V], ctypes.c_int),
             "star_decode_step_noalloc": ([P(StarShape), P(StarCache), V, V, V, V, I32, V, V, V], ctypes.c_int),
+            "star_encode_layers": ([P(StarShape), I32, P(StarCache), V, V, V, V, V, V, LAYER_FN, V, V], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -264,6 +271,37 @@ def star_decode_step_noalloc(shape, cache: PagedKVCache, q, k, v, pos, cur_len: 
                                           _ptr(k, "k", torch.bfloat16), _ptr(v, "v", torch.bfloat16),
                                           _ptr(pos, "pos", torch.int32), cur_len, _ptr(out, "out", torch.bfloat16),
                                           _ptr(lse_out, "lse_out", torch.float32), _stream(stream)))
+
+
+def star_encode_layers(shape, caches, pos_ctx, x, q, k, v, o, fn, stream=None):
+    """Multi-layer context encoding (star_encode_layers in star.h).
+
+    fn(layer, stage, x, q, k, v, o) enqueues the caller's work on the current stream:
+    stage STAR_LAYER_QKV writes q, k, v from x; stage STAR_LAYER_OUT updates x in place
+    from the attention output o.  caches: one PagedKVCache per layer.  An exception in
+    fn stops the call and is raised again here.
+    """
+    if isinstance(caches, PagedKVCache):
+        raise TypeError("caches must be a sequence of PagedKVCache, one per layer")
+    arr = (StarCache * len(caches))(*[c.c for c in caches])
+    raised = []
+
+    def trampoline(layer, stage, _in, _o0, _o1, _o2, _user, _stream_handle):
+        try:
+            fn(int(layer), int(stage), x, q, k, v, o)
+            return 0
+        except BaseException as e:  # re-raised after the C call returns
+            raised.append(e)
+            return 1
+
+    cb = LAYER_FN(trampoline)
+    rc = lib().star_encode_layers(ctypes.byref(shape), len(caches), arr, _ptr(pos_ctx, "pos_ctx", torch.int32),
+                                  _ptr(x, "x"), _ptr(q, "q", torch.bfloat16), _ptr(k, "k", torch.bfloat16),
+                                  _ptr(v, "v", torch.bfloat16), _ptr(o, "o", torch.bfloat16), cb, None,
+                                  _stream(stream))
+    if raised:
+        raise raised[0]
+    _check(rc)
 
 
 def star_device_status(stream=None) -> int:

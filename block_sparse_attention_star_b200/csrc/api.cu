@@ -343,6 +343,35 @@ int star_phase1_encode_anchored(const star_shape* shape, const star_cache* cache
   return STAR_OK;
 }
 
+int star_encode_layers(const star_shape* shape, int32_t n_layers, const star_cache* caches, const int32_t* pos_ctx,
+                       void* x, void* q, void* k, void* v, void* o, star_layer_fn fn, void* user,
+                       star_stream_t stream) {
+  int rc = check_shape(shape);
+  if (rc) return rc;
+  if (n_layers < 1) return fail(STAR_ERR_INVALID_ARG, "n_layers (%d) must be >= 1", n_layers);
+  if (!caches) return fail(STAR_ERR_INVALID_ARG, "caches is NULL");
+  if (!fn) return fail(STAR_ERR_INVALID_ARG, "fn is NULL");
+  if (!x) return fail(STAR_ERR_INVALID_ARG, "x is NULL");
+  STAR_REQUIRE_PTR(q, "q");
+  STAR_REQUIRE_PTR(k, "k");
+  STAR_REQUIRE_PTR(v, "v");
+  STAR_REQUIRE_PTR(o, "o");
+  STAR_REQUIRE_PTR4(pos_ctx, "pos_ctx");
+  for (int l = 0; l < n_layers; ++l) {
+    rc = check_cache(shape, &caches[l]);
+    if (rc) return rc;
+  }
+  for (int l = 0; l < n_layers; ++l) {
+    int cb = fn(l, STAR_LAYER_QKV, x, q, k, v, user, stream);
+    if (cb) return fail(STAR_ERR_CALLBACK, "layer callback returned %d (layer %d, q/k/v stage)", cb, l);
+    rc = star_phase1_encode(shape, &caches[l], q, k, v, pos_ctx, o, nullptr, 0, stream);
+    if (rc) return rc;
+    cb = fn(l, STAR_LAYER_OUT, o, x, nullptr, nullptr, user, stream);
+    if (cb) return fail(STAR_ERR_CALLBACK, "layer callback returned %d (layer %d, output stage)", cb, l);
+  }
+  return STAR_OK;
+}
+
 int star_phase2_partial(const star_shape* shape, const star_cache* cache, const void* q, const void* k, const void* v,
                         const int32_t* q_pos, int32_t T, float* o_part, float* lse_part, void* ws, size_t ws_bytes,
                         star_stream_t stream) {

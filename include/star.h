@@ -51,7 +51,8 @@ enum {
   STAR_ERR_ALIGNMENT = -3,        /* a pointer is not aligned as stated above */
   STAR_ERR_CAPACITY = -4,         /* page table / pool / workspace too small */
   STAR_ERR_CUDA = -5,             /* a CUDA runtime or driver call failed */
-  STAR_ERR_TIMEOUT = -6           /* a kernel gave up a bounded wait (see star_device_status) */
+  STAR_ERR_TIMEOUT = -6,          /* a kernel gave up a bounded wait (see star_device_status) */
+  STAR_ERR_CALLBACK = -7          /* a caller callback returned non-zero (star_encode_layers) */
 };
 
 /* Workspace query selectors. */
@@ -225,6 +226,34 @@ int star_decode_step(const star_shape* shape, const star_cache* cache, const voi
 int star_decode_step_noalloc(const star_shape* shape, const star_cache* cache, const void* q, const void* k,
                              const void* v, const int32_t* pos, int32_t cur_len, void* out, float* lse_out,
                              star_stream_t stream);
+
+/* Multi-layer context encoding ("仓库里的真实实现": every augmented block [a_1; c_i] runs
+ * the whole model forward on its own, and the anchor's part of every layer's KV is
+ * dropped).  The caller owns the model: for each layer the library calls `fn` twice,
+ * and `fn` enqueues the caller's own kernels (projections, residuals, MLP, ...) on
+ * `stream`:
+ *   fn(layer, STAR_LAYER_QKV, x, q, k, v, user, stream): q, k, v (pre-RoPE, the
+ *       layouts of star_phase1_encode) from the hidden states x;
+ *   fn(layer, STAR_LAYER_OUT, o, x, NULL, NULL, user, stream): the next hidden states
+ *       into x (in place) from the attention output o = star_phase1_encode(q, k, v).
+ * Between the two calls the library runs star_phase1_encode with layer's cache
+ * caches[layer].  The anchor is a prefix of block 1 with block 1's position ids, and
+ * attention is causal, so at every layer its hidden states, and its keys and values,
+ * are block 1's: one pass over the L real tokens per layer gives every block the
+ * anchor the pages recompute per host, exactly.  Anchor position ids other than
+ * block 1's would break that equality, so this call takes none.
+ * x: caller-owned device buffer of the hidden states (its layout is the caller's
+ * business; the library only passes it to fn).  q, o: bf16 [B][L][Hq][d]; k, v: bf16
+ * [B][L][Hkv][d], caller-owned scratch reused by every layer.  caches: n_layers
+ * caches (host array of star_cache), each as for star_phase1_encode.
+ * Errors: those of star_phase1_encode; CALLBACK if fn returns non-zero (the call stops
+ * there; work already enqueued stays enqueued). */
+enum { STAR_LAYER_QKV = 0, STAR_LAYER_OUT = 1 };
+typedef int (*star_layer_fn)(int32_t layer, int32_t stage, void* in, void* out0, void* out1, void* out2, void* user,
+                             star_stream_t stream);
+int star_encode_layers(const star_shape* shape, int32_t n_layers, const star_cache* caches, const int32_t* pos_ctx,
+                       void* x, void* q, void* k, void* v, void* o, star_layer_fn fn, void* user,
+                       star_stream_t stream);
 
 /* Tracing: when both are non-NULL (cudaEvent_t handles created by the caller),
  * every later call on this thread records `start_event` on its stream right

@@ -57,6 +57,9 @@ Parity status per function (the pins live in ``tests/test_oracle_pins.py``):
 * ``attend``/``phase2_partials``/``lse_merge``/``decode_step`` pinned: the merge
   equals brute-force softmax over the concatenated cache (library SDPA and
   scipy logsumexp); merge identities and overflow cases in closed form.
+* ``encode_layers`` pinned: equals the literal per-block forward (every augmented block
+  [anchor; c_i] through all layers on its own, anchor rows dropped), for a = b and a < b;
+  one block equals a textbook stack of causal attention layers.
 * ``kv_bytes_per_token``/``phase2_comm_bytes`` pinned: the pages' printed numbers.
 """
 
@@ -70,7 +73,7 @@ __all__ = [
     "round_to_bf16", "rope_inv_freq", "rope_angles", "apply_rope", "rope_bf16",
     "augmented_context", "block_map", "causal_attention", "attend", "phase1",
     "phase1_rows", "append_tail", "phase2_partials", "global_attention",
-    "lse_merge", "decode_step", "run_star", "kv_bytes_per_token",
+    "lse_merge", "decode_step", "run_star", "encode_layers", "kv_bytes_per_token",
     "phase2_comm_bytes",
 ]
 
@@ -448,6 +451,37 @@ def run_star(inp: dict, L: int, b: int, theta: float, with_phase1: bool = True, 
         else:
             out[k] = np.stack(vals)
     return out
+
+
+# ----------------------------------------------------------------------------
+# Several layers ([SA1] "仓库里的真实实现")
+# ----------------------------------------------------------------------------
+
+def encode_layers(x: np.ndarray, pos_ctx, b: int, theta: float, layers, anchor: int | None = None):
+    """Phase 1 of a stack of layers for one sequence, one pass over the L real tokens per layer.
+
+    [SA1] "仓库里的真实实现": every augmented block [a_1; c_i] runs the whole model forward
+    on its own (past_key_values=None), and the anchor's part of every layer's KV is
+    dropped.  The anchor is the first a tokens of c_1 with c_1's position ids and the
+    attention is causal, so its hidden states at every layer are c_1's first a rows;
+    the layer-by-layer pass below therefore takes the anchor's keys and values of each
+    layer from that layer's c_1 (through ``phase1``).  The pins check this against the
+    literal per-block forward.
+
+    x: hidden states [L, ...] (float64; the caller's layout).  layers: a list of
+    (qkv_fn, out_fn) per layer, the caller's model in float64: qkv_fn(x) -> q [L, Hq, d],
+    k, v [L, Hkv, d] (pre-RoPE, rounded as the caller rounds them); out_fn(x, o) -> the
+    next x, from the attention output o rounded to bf16 (the output type of Phase 1).
+    Returns the final x and, per layer, (o, cache K, cache V).
+    """
+    per_layer = []
+    for qkv_fn, out_fn in layers:
+        q, k, v = qkv_fn(x)
+        o, ck, cv = phase1(q, k, v, pos_ctx, b, theta, anchor)
+        o = round_to_bf16(o)
+        per_layer.append((o, ck, cv))
+        x = out_fn(x, o)
+    return x, per_layer
 
 
 # ----------------------------------------------------------------------------

@@ -12,6 +12,7 @@ from .configs import CONFIGS, Workload, get_config  # noqa: F401
 from .gen import (  # noqa: F401
     STREAM_IDS,
     gaussian_bf16,
+    layer_inputs,
     make_inputs,
     peaky_rows,
     splitmix64_reference,

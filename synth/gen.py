@@ -43,6 +43,7 @@ STREAM_IDS = {
     "q_dec": 7, "k_dec": 8, "v_dec": 9,
     "peaky": 10,
     "anchor": 11,
+    "x_layers": 12, "w_layers": 13,
 }
 
 _CHUNK = 1 << 24
@@ -155,6 +156,29 @@ def anchor_positions(wl: Workload, device="cpu") -> torch.Tensor:
     span = (idx % (n - 1) + 1) * b - a + 1          # block i = idx % (n-1) + 1
     off = (u % span).view(B, n - 1, 1)
     return (off + torch.arange(a, dtype=torch.int64, device=device)).to(torch.int32).contiguous()
+
+
+def layer_inputs(seed: int, n_layers: int, B: int, L: int, hidden: int, q_width: int, kv_width: int,
+                 device="cpu") -> tuple[torch.Tensor, list[tuple[torch.Tensor, ...]]]:
+    """Hidden states and random per-layer weights for the multi-layer tests.
+
+    x0: [B, L, hidden] N(0, 1) bf16.  Per layer: Wq [hidden, q_width], Wk and Wv
+    [hidden, kv_width], Wo [q_width, hidden], N(0, 1) bf16 draws times a power of two
+    close to 1/sqrt(fan-in) (exact in bf16), drawn in that order from one stream.
+    """
+    x0 = gaussian_bf16(seed, STREAM_IDS["x_layers"], (B, L, hidden), device)
+    shapes = [(hidden, q_width), (hidden, kv_width), (hidden, kv_width), (q_width, hidden)]
+    per = sum(a * b for a, b in shapes)
+    flat = gaussian_bf16(seed, STREAM_IDS["w_layers"], (n_layers * per,), device)
+    ws, off = [], 0
+    for _ in range(n_layers):
+        mats = []
+        for fan_in, fan_out in shapes:
+            scale = 2.0 ** -round(math.log2(math.sqrt(fan_in)))
+            mats.append((flat[off:off + fan_in * fan_out].view(fan_in, fan_out) * scale).contiguous())
+            off += fan_in * fan_out
+        ws.append(tuple(mats))
+    return x0, ws
 
 
 def make_inputs(wl: Workload, device="cpu", parts=("ctx", "query", "dec")) -> dict[str, torch.Tensor]:

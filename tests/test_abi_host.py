@@ -4,6 +4,7 @@ every symbol the header declares, and validates shapes and capacities."""
 import ctypes
 
 import pytest
+import torch
 
 import block_sparse_attention_star_b200 as star
 from synth import CONFIGS
@@ -121,3 +122,32 @@ def test_phase2_and_decode_workspaces_are_checked_before_any_launch():
     rc = lib.star_decode_step(ctypes.byref(sh), ctypes.byref(cache), p, p, p, p, sh.L, p, None, p, need_d - 256,
                               None)
     assert rc == star.STAR_ERR_CAPACITY
+
+
+def test_encode_layers_callback_marshalling_without_a_launch():
+    """star_encode_layers validates its arguments, then calls the caller's callback before
+    any launch: an exception raised there stops the call (STAR_ERR_CALLBACK in C) and is
+    raised again by the binding, with no CUDA call made."""
+    sh = _shape(L=512, b=256)
+    max_pages = star.star_pages_needed(sh)
+
+    class FakeCache:  # never dereferenced: the call stops in the first callback
+        c = star.StarCache(k_pool=256, v_pool=256, page_table=256, max_pages=max_pages, num_pages=1)
+
+    x = torch.zeros(16, dtype=torch.bfloat16)
+    t = torch.zeros(16, dtype=torch.bfloat16)
+    pos = torch.zeros(16, dtype=torch.int32)
+    calls = []
+
+    def fn(layer, stage, *tensors):
+        calls.append((layer, stage, len(tensors)))
+        raise KeyError("model failed")
+
+    with pytest.raises(KeyError):
+        star.star_encode_layers(sh, [FakeCache(), FakeCache()], pos, x, t, t, t, t, fn, stream=0)
+    assert calls == [(0, star.STAR_LAYER_QKV, 5)]
+    assert "callback" in star.lib().star_last_error().decode()
+    with pytest.raises(star.StarError) as e:  # a NULL callback is rejected up front
+        star._check(star.lib().star_encode_layers(ctypes.byref(sh), 1, ctypes.byref(FakeCache.c), None, None, None,
+                                                  None, None, None, star.LAYER_FN(), None, None))
+    assert e.value.code == star.STAR_ERR_INVALID_ARG
