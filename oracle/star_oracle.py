@@ -35,7 +35,16 @@ projections):
    including its own K/V ([SA2] abstract: query and response tokens attend to all
    prior cached tokens).
 
-Readings where the pages are silent are listed in the design doc's readings table.
+Readings taken where the pages are silent or disagree: softmax scale 1/sqrt(d)
+(the one of [SA1] "Phase 2: 局部注意力与本地统计量"); plain RoPE with theta =
+500000, rotate-half pairing and no frequency scaling; the angle exact in float64;
+roped Q and K rounded once to bf16; the cache holds roped K and raw V; causality by
+cache index (c_i rows see the whole anchor, anchor rows only the anchor); GQA head
+map kv = h // (Hq/Hkv); partials in float64 here (float32 on the GPU) with the final
+O rounded to bf16; a partial with a non-finite LSE contributes nothing and a row with
+none gives O = 0, LSE = -inf; the merge in max-subtracted log-sum-exp form; the
+query and generated tokens' K/V at the tail of the last block, causal among
+themselves, a decode token attending to itself.
 
 Parity status per function (the pins live in ``tests/test_oracle_pins.py``):
 
