@@ -146,6 +146,18 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # The CUDA path
 # ---------------------------------------------------------------------------
+def launches_per_step(star, shape, wl, anchor_ids: bool) -> int:
+    """Library kernel launches in one step.  Phase 1: RoPE + KV append, tail zero-fill,
+    RoPE(Q), attention (+ the anchor keys at caller ids).  Phase 2: query KV append,
+    RoPE(Q), attention (+ the chunk merge when blocks are split into chunks, i.e. when
+    the workspace holds more than RoPE(Q)).  The query merge.  Per decode step: the
+    decode kernel (one launch: its chunking keeps the items within one launch) and its
+    merge."""
+    q_bytes = -(-wl.B * wl.T * wl.Hq * wl.d * 2 // 256) * 256
+    chunked = star.star_workspace_size(shape, star.STAR_OP_PHASE2, wl.T) > q_bytes
+    return (4 + (1 if anchor_ids else 0)) + (3 + (1 if chunked else 0)) + 1 + 2 * wl.S
+
+
 def workload_config(wl, world):
     """The `config` object of the JSON line (the same for both arms)."""
     return {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d, "L": wl.L, "b": wl.b,
@@ -182,8 +194,7 @@ class StarRun:
         self.lse_q = torch.empty((wl.B, wl.T, wl.Hq), dtype=torch.float32, device=device)
         self.o_dec = torch.empty((wl.S, wl.B, 1, wl.Hq, wl.d), dtype=torch.bfloat16, device=device)
         self.lse_dec = torch.empty((wl.S, wl.B, wl.Hq), dtype=torch.float32, device=device)
-        cpb_ws = star.star_workspace_size(self.shape, star.STAR_OP_PHASE2, wl.T)
-        self.launches_per_step = 3 + 2 + (1 if cpb_ws > 0 else 0) + 1 + 3 * wl.S
+        self.launches_per_step = launches_per_step(star, self.shape, wl, anchor_ids="anchor_pos" in self.inp)
 
     def step(self, ev=None):
         """One pass of the hot path.  ev: optional dict of (start, stop) event lists to record."""
