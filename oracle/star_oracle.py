@@ -66,6 +66,12 @@ Parity status per function (the pins live in ``tests/test_oracle_pins.py``):
 * ``attend``/``phase2_partials``/``lse_merge``/``decode_step`` pinned: the merge
   equals brute-force softmax over the concatenated cache (library SDPA and
   scipy logsumexp); merge identities and overflow cases in closed form.
+* ``run_star`` (the whole path) pinned in ``tests/test_oracle_path.py``: with one block it
+  equals one index-causal library SDPA over the concatenated [c, q, gen]; with n > 1 its
+  query and decode outputs and LSEs equal library SDPA over the independently roped,
+  explicitly concatenated cache, its Phase-1 rows the full-length Star mask, its partials
+  SDPA over each block's keys; per-sequence lengths likewise; decode steps that do not
+  carry the cache forward, and a query tail placed before the context, are caught.
 * ``encode_layers`` pinned: equals the literal per-block forward (every augmented block
   [anchor; c_i] through all layers on its own, anchor rows dropped), for a = b and a < b;
   one block equals a textbook stack of causal attention layers.
