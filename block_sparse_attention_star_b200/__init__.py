@@ -39,6 +39,7 @@ STAR_ERR_TIMEOUT = -6
 STAR_ERR_CALLBACK = -7
 STAR_LAYER_QKV, STAR_LAYER_OUT = 0, 1
 STAR_OP_PHASE1, STAR_OP_PHASE2, STAR_OP_DECODE, STAR_OP_PHASE1_ANCHOR = 1, 2, 3, 4
+STAR_DEBUG_SKIP_FIRST_LOAD = 1
 
 
 class StarError(RuntimeError):
@@ -110,6 +111,7 @@ def lib() -> ctypes.CDLL:
             "star_set_trace_events": ([V, V], ctypes.c_int),
             "star_decode_step_noalloc": ([P(StarShape), P(StarCache), V, V, V, V, I32, V, V, V], ctypes.c_int),
             "star_encode_layers": ([P(StarShape), I32, P(StarCache), V, V, V, V, V, V, LAYER_FN, V, V], ctypes.c_int),
+            "star_debug_set": ([ctypes.c_uint64, I32], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -309,6 +311,12 @@ def star_device_status(stream=None) -> int:
     rc = lib().star_device_status(_stream(stream), ctypes.byref(code))
     _check(rc)
     return code.value
+
+
+def star_debug_set(wait_limit_ns: int = 0, flags: int = 0) -> None:
+    """Failure-detection test hook: the bounded waits' limit (0 = the default 2 s) and
+    debug flags (STAR_DEBUG_SKIP_FIRST_LOAD) for later attention and decode launches."""
+    _check(lib().star_debug_set(int(wait_limit_ns), int(flags)))
 
 
 def workspace(shape: StarShape, op: int, T: int = 0, device="cuda") -> torch.Tensor:

@@ -41,12 +41,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 
-int num_sms() {
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
-  return sms > 0 ? sms : 148;
-}
+int num_sms() { return star::current_device_sm_count(); }
 
 int check_shape(const star_shape* s) {
   if (!s) return fail(STAR_ERR_INVALID_ARG, "shape is NULL");
@@ -199,6 +194,20 @@ size_t decode_ws_bytes(const star_shape* s) {
 
 namespace star {
 int set_last_error(int code, const char* msg) { return fail(code, "%s", msg); }
+
+int current_device_sm_count() {
+  static std::atomic<int> cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 64) {
+    const int c = cached[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) return 148;
+  if (dev >= 0 && dev < 64) cached[dev].store(sms, std::memory_order_relaxed);
+  return sms;
+}
 }  // namespace star
 
 extern "C" {
@@ -525,7 +534,7 @@ int star_device_status(star_stream_t stream, int32_t* status_out) {
   int code = 0;
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   cudaError_t (*readers[])(int*) = {star::read_and_clear_error_attn, star::read_and_clear_error_decode,
-                                   star::read_and_clear_error_rope};
+                                   star::read_and_clear_error_rope, star::read_and_clear_error_merge};
   for (auto rd : readers) {
     if (e != cudaSuccess) break;
     int c = 0;
@@ -535,8 +544,19 @@ int star_device_status(star_stream_t stream, int32_t* status_out) {
   if (status_out) *status_out = code;
   if (e != cudaSuccess) return cuda_fail(e, "device status");
   if (code == star::kDevBadPage) return fail(STAR_ERR_CAPACITY, "a page-table entry was outside [0, num_pages)");
+  if (code == star::kDevBadPartial)
+    return fail(STAR_ERR_INVALID_ARG, "a merged partial had a NaN or +inf log-sum-exp (it was skipped)");
   if (code != 0) return fail(STAR_ERR_TIMEOUT, "a kernel gave up a bounded wait (code %d)", code);
   return STAR_OK;
+}
+
+int star_debug_set(uint64_t wait_limit_ns, int32_t flags) {
+  if (flags & ~STAR_DEBUG_SKIP_FIRST_LOAD) return fail(STAR_ERR_INVALID_ARG, "unknown debug flags 0x%x", flags);
+  const unsigned long long limit = wait_limit_ns ? wait_limit_ns : star::kDefaultWaitLimitNs;
+  const int dev_flags = (flags & STAR_DEBUG_SKIP_FIRST_LOAD) ? star::kDebugSkipFirstLoad : 0;
+  cudaError_t e = star::set_debug_attn(limit, dev_flags);
+  if (e == cudaSuccess) e = star::set_debug_decode(limit, dev_flags);
+  return e == cudaSuccess ? STAR_OK : cuda_fail(e, "debug settings");
 }
 
 }  // extern "C"

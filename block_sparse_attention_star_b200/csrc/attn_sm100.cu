@@ -278,6 +278,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t kcnt = 0, vcnt = 0;
       bool ok = true;
+      // Test hook: CTA 0 issues no first K load, so every role's bounded wait runs out.
+      const bool skip_first = blockIdx.x == 0 && (g_debug_flags & kDebugSkipFirstLoad);
       for (int idx = blockIdx.x; idx < p.num_items && ok; idx += gridDim.x) {
         const Item it = decode_item<MODE>(p, idx);
         if (it.skip) continue;
@@ -291,15 +293,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int s = kcnt % NSK;
             ok = mbar_wait(&k_empty[s], ((kcnt / NSK) & 1) ^ 1, kDevTimeoutProducer);
             if (!ok) break;
-            mbar_arrive_expect_tx(&k_full[s], S::kTile);
             uint8_t* dst = smem + S::kK + s * S::kTile;
-            if (MODE == 0 && p.anchor_k_on && j < it.a_tiles) {
+            if (skip_first && kcnt == 0) {
+              // (test hook) no arrival and no load: k_full[0] never completes
+            } else if (MODE == 0 && p.anchor_k_on && j < it.a_tiles) {
+              mbar_arrive_expect_tx(&k_full[s], S::kTile);
               // The anchor's keys roped at the caller's ids: [B][n-1][Hkv][a][d], block it.part.
 #pragma unroll
               for (int h = 0; h < D / 64; ++h)
                 tma_load_4d(dst + h * (kKeys * 128), &tmKA, &k_full[s], h * 64, j * kKeys, it.g,
                             it.bi * (p.n - 1) + it.part - 1);
             } else {
+              mbar_arrive_expect_tx(&k_full[s], S::kTile);
 #pragma unroll
               for (int h = 0; h < D / 64; ++h)
                 tma_load_4d(dst + h * (kKeys * 128), &tmK, &k_full[s], h * 64, slot, it.g, page);
@@ -740,16 +745,10 @@ cudaError_t launch_typed(const AttnLaunch& a, const Params& p, const CUtensorMap
   constexpr int NSV = (D == 128) ? 2 : 4;
   using S = Smem<D, MODE, NSK, NSV>;
   auto kern = star_attn_kernel<D, MODE, NSK, NSV>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int grid = std::min(p.num_items, sms);
+  static std::atomic<unsigned long long> smem_opted_in{0};
+  cudaError_t e = opt_in_dynamic_smem(reinterpret_cast<const void*>(kern), S::kBytes, smem_opted_in);
+  if (e != cudaSuccess) return e;
+  const int grid = std::min(p.num_items, current_device_sm_count());
   if (grid <= 0) return cudaSuccess;
   kern<<<grid, kThreads, S::kBytes, st>>>(mk, mv, mq, mka, p);
   return cudaGetLastError();
@@ -819,5 +818,6 @@ cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t st, const char** 
 }
 
 cudaError_t read_and_clear_error_attn(int* code) { return read_and_clear_tu_error(code); }
+cudaError_t set_debug_attn(unsigned long long wait_limit_ns, int flags) { return set_tu_debug(wait_limit_ns, flags); }
 
 }  // namespace star

@@ -38,8 +38,19 @@ enum DeviceError : int {
   kDevTimeoutMma = 2,
   kDevTimeoutSoftmax = 3,
   kDevBadPage = 4,
+  kDevBadPartial = 5,   // a merged partial had a NaN or +inf LSE (skipped, like an empty one)
 };
 static __device__ int g_device_error = 0;
+
+// Failure-detection test hooks, one copy per translation unit like the error word:
+// the bounded waits' limit (nanoseconds), and debug flags (kDebugSkipFirstLoad: the
+// producer of CTA 0 issues no first K tile load, so the barrier of that stage never
+// completes and every role's bounded wait runs out; nothing asynchronous is left in
+// flight).  Both are set from the host between launches (star_debug_set).
+constexpr unsigned long long kDefaultWaitLimitNs = 2000000000ull;
+constexpr int kDebugSkipFirstLoad = 1;
+static __device__ unsigned long long g_wait_limit_ns = kDefaultWaitLimitNs;
+static __device__ int g_debug_flags = 0;
 
 __device__ __forceinline__ void record_error(int code) { atomicCAS(&g_device_error, 0, code); }
 
@@ -50,6 +61,13 @@ static inline cudaError_t read_and_clear_tu_error(int* code) {
   if (e != cudaSuccess) return e;
   const int zero = 0;
   return cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+}
+
+// Host: set this translation unit's wait limit and debug flags.
+static inline cudaError_t set_tu_debug(unsigned long long wait_limit_ns, int flags) {
+  cudaError_t e = cudaMemcpyToSymbol(g_wait_limit_ns, &wait_limit_ns, sizeof(wait_limit_ns));
+  if (e != cudaSuccess) return e;
+  return cudaMemcpyToSymbol(g_debug_flags, &flags, sizeof(flags));
 }
 
 // cos and sin of pos * inv_freq in float64 (argument reduced modulo 2*pi first).
@@ -106,15 +124,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete.  Gives up after
-// `limit_ns` (checked every 64 polls), records `err` and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int err,
-                                          uint64_t limit_ns = 2000000000ull) {
+// Wait for the phase with the given parity to complete.  Gives up after the
+// translation unit's limit (2 s unless a test shortened it; checked every 64
+// polls), records `err` and returns false.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int err) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0 && globaltimer_ns() - t0 > limit_ns) {
+    if ((it & 63u) == 0 && globaltimer_ns() - t0 > g_wait_limit_ns) {
       record_error(err);
       return false;
     }

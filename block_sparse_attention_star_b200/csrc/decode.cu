@@ -348,6 +348,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t kc = 0;
       bool ok = true;
+      // Test hook: CTA 0 issues no first K load, so every role's bounded wait runs out.
+      const bool skip_first = blockIdx.x == 0 && (g_debug_flags & kDebugSkipFirstLoad);
       for (int ii = 0; ii < n_my && ok; ++ii) {
         const DecItem it = dec_item(p, first + ii * gridDim.x);
         for (int t = 0; t < it.ntiles && ok; ++t, ++kc) {
@@ -367,11 +369,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t ph = ((kc / NST) & 1) ^ 1;
           ok = mbar_wait(&k_empty[s], ph, kDevTimeoutProducer);
           if (!ok) break;
-          mbar_arrive_expect_tx(&k_full[s], S::kTile);
+          if (!(skip_first && kc == 0)) {  // (test hook) no arrival and no load: k_full[0] never completes
+            mbar_arrive_expect_tx(&k_full[s], S::kTile);
 #pragma unroll
-          for (int h = 0; h < D / 64; ++h)
-            tma_load_4d(smem + S::kK + s * S::kTile + h * (kTileKeys * 128), &tmK, &k_full[s], h * 64, slot, it.g,
-                        page);
+            for (int h = 0; h < D / 64; ++h)
+              tma_load_4d(smem + S::kK + s * S::kTile + h * (kTileKeys * 128), &tmK, &k_full[s], h * 64, slot, it.g,
+                          page);
+          }
           ok = mbar_wait(&v_empty[s], ph, kDevTimeoutProducer);
           if (!ok) break;
           mbar_arrive_expect_tx(&v_full[s], S::kTile);
@@ -615,28 +619,14 @@ bool make_tile_map(CUtensorMap* map, void* pool, int d, int P, int Hkv, int num_
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int num_sms_cached() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
-
 template <int D, int G>
 cudaError_t launch_dg(DecParams p, const CUtensorMap& mk, const CUtensorMap& mv, int total_items, cudaStream_t st) {
   using S = DecSmem<D>;
   auto kern = decode_kernel<D, G>;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kBytes);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
-  const int grid = std::min(total_items, num_sms_cached());
+  static std::atomic<unsigned long long> smem_opted_in{0};
+  cudaError_t e0 = opt_in_dynamic_smem(reinterpret_cast<const void*>(kern), S::kBytes, smem_opted_in);
+  if (e0 != cudaSuccess) return e0;
+  const int grid = std::min(total_items, current_device_sm_count());
   // Each launch covers at most kMaxItems items per CTA.
   for (int base = 0; base < total_items; base += grid * kMaxItems) {
     p.item_base = base;
@@ -650,6 +640,7 @@ cudaError_t launch_dg(DecParams p, const CUtensorMap& mk, const CUtensorMap& mv,
 }  // namespace
 
 cudaError_t read_and_clear_error_decode(int* code) { return read_and_clear_tu_error(code); }
+cudaError_t set_debug_decode(unsigned long long wait_limit_ns, int flags) { return set_tu_debug(wait_limit_ns, flags); }
 
 int decode_num_chunks(int n_keys, int chunk) { return (n_keys + chunk - 1) / chunk; }
 

@@ -5,9 +5,27 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <utility>
 
 namespace star {
+
+// A kernel that uses more than 48 KB of dynamic shared memory must opt in once per
+// device.  `done` (one per kernel) remembers the devices (ordinals < 64) already set,
+// so a process that drives several GPUs opts in on each of them.
+inline cudaError_t opt_in_dynamic_smem(const void* kern, int bytes, std::atomic<unsigned long long>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
+  return e;
+}
+
+// SM count of the current device (looked up once per device; 148 if the query fails).
+int current_device_sm_count();
 
 // A launch with programmatic stream serialization: the kernel may start while the
 // previous kernel in the stream drains, and waits (griddepcontrol.wait) before it
@@ -129,5 +147,10 @@ int set_last_error(int code, const char* msg);
 cudaError_t read_and_clear_error_attn(int* code);
 cudaError_t read_and_clear_error_decode(int* code);
 cudaError_t read_and_clear_error_rope(int* code);
+cudaError_t read_and_clear_error_merge(int* code);
+
+// --- failure-detection test hooks (per kernel file; see common.cuh) -------------
+cudaError_t set_debug_attn(unsigned long long wait_limit_ns, int flags);
+cudaError_t set_debug_decode(unsigned long long wait_limit_ns, int flags);
 
 }  // namespace star

@@ -5,8 +5,11 @@
 //
 // With m = max_i LSE_i over the partials whose LSE is finite,
 //   LSE = m + log(sum_i exp(LSE_i - m)),   O = sum_i exp(LSE_i - LSE) O_i.
-// A partial with a non-finite LSE (an empty block: -inf) contributes nothing;
-// a row with no finite partial gives O = 0, LSE = -inf.
+// A partial with a non-finite LSE (an empty block: -inf) contributes nothing,
+// and its O is never read into the sum (an empty partial's O may be 0/0); a row
+// with no finite partial gives O = 0, LSE = -inf.  A NaN or +inf LSE cannot come
+// from a correct partial: it is skipped the same way and also recorded in the
+// device error word (kDevBadPartial), which star_device_status reports.
 //
 // One warp per output row; each lane owns d/32 consecutive columns (one
 // 16-byte load per partial at d = 128).  The kernel is latency-bound at decode
@@ -67,9 +70,13 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(int parts_per_group, lon
 
   // LSE statistics: online (max, sum) over the lane's partials, then across lanes.
   float m = -INFINITY, s = 0.f;
+  bool bad = false;
   for (int i = lane; i < np; i += 32) {
     const float li = __ldg(lb + (size_t)i * rows);
-    if (!isfinite(li)) continue;
+    if (!isfinite(li)) {
+      bad |= !(li == -INFINITY);
+      continue;
+    }
     if (li > m) {
       s = s * expf(m - li) + 1.f;
       m = li;
@@ -85,6 +92,7 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(int parts_per_group, lon
     m = mm;
   }
   const float lse = (m == -INFINITY) ? -INFINITY : m + logf(s);
+  if (bad) record_error(kDevBadPartial);
 
   float acc[PER];
 #pragma unroll
@@ -105,7 +113,7 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(int parts_per_group, lon
 #pragma unroll
       for (int j = 0; j < kBatch; ++j) {
         const float wj = __shfl_sync(0xffffffffu, w, j);
-        if (base + j < np) Cols<D>::fma(acc, wj, v[j]);
+        if (base + j < np && wj != 0.f) Cols<D>::fma(acc, wj, v[j]);
       }
     }
   }
@@ -123,6 +131,8 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(int parts_per_group, lon
 }
 
 }  // namespace
+
+cudaError_t read_and_clear_error_merge(int* code) { return read_and_clear_tu_error(code); }
 
 cudaError_t launch_lse_merge(int groups, int parts_per_group, int64_t rows, int d, const float* o_in,
                              const float* lse_in, void* o_out, bool out_bf16, float* lse_out, cudaStream_t st) {

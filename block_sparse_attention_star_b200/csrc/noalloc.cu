@@ -24,8 +24,9 @@
 
 namespace {
 
-// 16 MiB: the partials of a decode step over a one-million-token cache with 32
-// query heads (513 chunks x 32 rows x 129 floats) fit with room to spare.
+// 16 MiB.  The decode step keeps at most 8 work items per CTA, so its chunk
+// partials are bounded by the item count, not by the cache length: 0.61 MB for the
+// Llama-3.1-8B shapes at 32K, 128K and 1M tokens, 2.4 MB for two 70B sequences.
 constexpr size_t kNoAllocScratchBytes = 16u << 20;
 constexpr int kMaxDevices = 64;
 
@@ -35,7 +36,9 @@ std::mutex g_lock;
 void* g_scratch_addr[kMaxDevices] = {nullptr};
 
 // Device address of the scratch array on the current device (looked up once).
-int scratch_for_current_device(void** out, char* why, size_t why_len) {
+// The lookup is not allowed while `stream` is being captured into a CUDA graph, so
+// a first call made during a capture is refused with a message instead.
+int scratch_for_current_device(cudaStream_t stream, void** out, char* why, size_t why_len) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) {
@@ -48,6 +51,19 @@ int scratch_for_current_device(void** out, char* why, size_t why_len) {
   }
   std::lock_guard<std::mutex> g(g_lock);
   if (!g_scratch_addr[dev]) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    e = cudaStreamIsCapturing(stream, &cap);
+    if (e != cudaSuccess) {
+      snprintf(why, why_len, "cudaStreamIsCapturing: %s", cudaGetErrorString(e));
+      return STAR_ERR_CUDA;
+    }
+    if (cap != cudaStreamCaptureStatusNone) {
+      snprintf(why, why_len,
+               "the first star_decode_step_noalloc call on device %d was made during stream capture; make one "
+               "call on this device before capturing",
+               dev);
+      return STAR_ERR_INVALID_ARG;
+    }
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || p == nullptr) {
@@ -78,7 +94,7 @@ extern "C" int star_decode_step_noalloc(const star_shape* shape, const star_cach
     return star::set_last_error(STAR_ERR_CAPACITY, g_why);
   }
   void* scratch = nullptr;
-  rc = scratch_for_current_device(&scratch, g_why, sizeof(g_why));
+  rc = scratch_for_current_device((cudaStream_t)stream, &scratch, g_why, sizeof(g_why));
   if (rc != STAR_OK) return star::set_last_error(rc, g_why);
   // Every partial the merge reads is written by the same call first, so nothing in
   // the array has to start at zero.

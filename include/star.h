@@ -217,7 +217,8 @@ int star_decode_step(const star_shape* shape, const star_cache* cache, const voi
  * Scratch: a 16 MiB device array built into the library (every GPU that loads the
  * library holds it until the process exits).  The first call made on a device
  * looks up that array's device address with cudaGetSymbolAddress, so make that
- * first call before any stream capture.  All calls share the one array and a call
+ * first call before any stream capture (a first call made while `stream` is being
+ * captured is refused with STAR_ERR_INVALID_ARG).  All calls share the one array and a call
  * writes every value it later reads, so nothing has to be cleared between calls,
  * but calls whose kernels overlap on the GPU (other streams, other threads) race
  * on it: serialise them.  No device memory is allocated or freed.
@@ -263,11 +264,27 @@ int star_encode_layers(const star_shape* shape, int32_t n_layers, const star_cac
  * Errors: INVALID_ARG if exactly one is NULL. */
 int star_set_trace_events(void* start_event, void* stop_event);
 
-/* Synchronises `stream`, then reads and clears the device error word that the
- * kernels set when a bounded wait runs out or a page-table entry is out of range.
- * *status_out receives the raw code (0 = none).  Returns STAR_ERR_TIMEOUT if a wait
- * ran out, STAR_ERR_CAPACITY for a bad page, STAR_ERR_CUDA if the stream failed. */
+/* Synchronises `stream`, then reads and clears the device error words that the
+ * kernels set when a bounded wait runs out, a page-table entry is out of range, or
+ * a merged partial carries a NaN or +inf log-sum-exp.  *status_out receives the raw
+ * code (0 = none; 1-3 a wait that ran out, 4 a bad page, 5 a bad partial).  Returns
+ * STAR_ERR_TIMEOUT if a wait ran out, STAR_ERR_CAPACITY for a bad page,
+ * STAR_ERR_INVALID_ARG for a bad partial, STAR_ERR_CUDA if the stream failed. */
 int star_device_status(star_stream_t stream, int32_t* status_out);
+
+/* Failure-detection test hook.  The Star Attention pages have no counterpart to
+ * this call: it lets a test watch the kernels' bounded waits give up without
+ * faulting or hanging the GPU.  wait_limit_ns: how long any mbarrier wait in the
+ * attention and decode kernels may last before the kernel records
+ * STAR_ERR_TIMEOUT's code and returns (0 restores the default of 2 s).  flags:
+ * STAR_DEBUG_SKIP_FIRST_LOAD makes CTA 0's producer of every later attention and
+ * decode launch issue no first K-tile load, so the barrier of that stage never
+ * completes, every role's bounded wait runs out, and nothing asynchronous is left
+ * in flight (0 = normal operation).  The settings hold for the current device
+ * until changed; call it between launches, never while kernels run.
+ * Errors: INVALID_ARG (unknown flag), CUDA. */
+enum { STAR_DEBUG_SKIP_FIRST_LOAD = 1 };
+int star_debug_set(uint64_t wait_limit_ns, int32_t flags);
 
 #ifdef __cplusplus
 }

@@ -117,10 +117,15 @@ def test_lse_merge_edge_cases():
         L[1, :50] = -np.inf                  # empty blocks
         L[:, 60] = -np.inf                   # a row with no usable partial
         L[0, 70:80] = 1e4                    # differences far beyond exp's range
-        L[2, 80:90] = np.nan                 # filtered like an empty block
+        L[2, 80:90] = np.nan                 # filtered like an empty block, and reported
+        O[1, :50] = np.nan                   # an empty partial's O (0/0) must not leak into the sum
         out = torch.empty((rows, d), dtype=torch.bfloat16, device="cuda")
         lse = torch.empty(rows, dtype=torch.float32, device="cuda")
         star.star_lse_merge(n, rows, d, torch.from_numpy(O).cuda(), torch.from_numpy(L).cuda(), out, lse)
+        with pytest.raises(star.StarError) as e:
+            star.star_device_status()
+        assert e.value.code == star.STAR_ERR_INVALID_ARG and "NaN or +inf" in str(e.value)
+        assert star.star_device_status() == 0          # read and cleared
         ref_o, ref_l = oracle.lse_merge(O.astype(np.float64), L.astype(np.float64))
         h = H()
         h.assert_out(out, ref_o, "merge O")
@@ -128,6 +133,11 @@ def test_lse_merge_edge_cases():
         assert np.isneginf(g[60]) and np.all(out[60].float().cpu().numpy() == 0)
         fin = np.isfinite(ref_l)
         assert np.all(np.abs(g[fin] - ref_l[fin]) <= 1e-3 * np.maximum(1.0, np.abs(ref_l[fin]) / 1e3))
+        # Without the NaN partials (-inf and huge differences only) nothing is reported.
+        L2 = np.where(np.isnan(L), -np.inf, L).astype(np.float32)
+        star.star_lse_merge(n, rows, d, torch.from_numpy(O).cuda(), torch.from_numpy(L2).cuda(), out, lse)
+        assert star.star_device_status() == 0
+        assert torch.isfinite(out.float()).all()
 
 
 def test_invalid_arguments_launch_nothing():
