@@ -14,8 +14,10 @@ timed region.
 
 Multi-GPU (torchrun): every rank runs its own independent sequence batch (the
 path partitions by sequence; no collective on the data path); time is the max
-over ranks.  `--impl reference` times the CPU oracle (float64 numpy) on a
-bounded sample of the same workload on the host cores.
+over ranks.  `--impl reference` times the CPU oracle (float64 numpy) on bounded
+samples of the same workload's step on the host cores and reports the whole step
+extrapolated from them (same metric and unit); `--oracle-full` times the whole
+oracle on a small workload.
 """
 
 from __future__ import annotations
@@ -51,6 +53,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=8, help="Phase-1 rows per block in the oracle sample")
+    ap.add_argument("--oracle-full", action="store_true",
+                    help="time the whole CPU oracle on the full workload (small workloads only) and exit")
     ap.add_argument("--layers", type=int, default=0,
                     help="time N layers of context encoding (star_encode_layers, random projections) instead")
     return ap.parse_args()
@@ -213,7 +217,11 @@ class StarRun:
                               wl.T, self.o_part, self.lse_part, self.ws2)
         if ev:
             s.star_set_trace_events(None, None)
+        if ev and "merge" in ev:
+            ev["merge"][0].record()
         s.star_lse_merge(self.shape.n, wl.B * wl.T * wl.Hq, wl.d, self.o_part, self.lse_part, self.o_q, self.lse_q)
+        if ev and "merge" in ev:
+            ev["merge"][1].record()
         # ev["dec_span"] brackets the S decode steps with nothing between their launches;
         # ev["dec"] (a separate instrumented step) brackets every decode attention kernel.
         if ev and "dec_span" in ev:
@@ -262,6 +270,31 @@ def max_over_ranks(value: float, device) -> float:
 def job_value(world: int, ctx_tokens: int, ms_per_step: float) -> float:
     """Whole-job context tokens per second: every rank encodes its batch's context each step."""
     return world * ctx_tokens / (ms_per_step * 1e-3)
+
+
+def phase2_roofline(wl, n, ms, peaks):
+    """Phase-2 query partials (RoPE(Q) pre-pass + attention kernel) against both bounds: the
+    query rows' products over every cached key (flop) and one read of the cache, the query and
+    the per-block partials written (bytes).  The roofline time is the larger of the two."""
+    T, d, Hq, Hkv = wl.T, wl.d, wl.Hq, wl.Hkv
+    lens = [wl.ctx_len(bi) for bi in range(wl.B)]
+    flop = sum(4.0 * d * Hq * T * (Ls + (T + 1) / 2.0) for Ls in lens)
+    byts = sum((Ls + T) * Hkv * d * 2 * 2 for Ls in lens) + wl.B * T * Hq * d * 2 + n * wl.B * T * Hq * (d + 1) * 4
+    t_flop = flop / (peaks["bf16"] * 1e12)
+    t_byte = byts / (peaks["hbm_gbs"] * 1e9)
+    sec = ms * 1e-3
+    return {"attn_ms": ms, "flop": flop, "bytes": byts, "tflops": flop / sec / 1e12, "gbs": byts / sec / 1e9,
+            "frac_tensor": t_flop / sec, "frac_hbm": t_byte / sec, "bound": "tensor" if t_flop >= t_byte else "hbm",
+            "frac": max(t_flop, t_byte) / sec, "peaks": f"{peaks['kind']} bf16 burst {peaks['bf16']} TF/s, "
+                                                       f"HBM {peaks['hbm_gbs']} GB/s"}
+
+
+def merge_roofline(rows, n, d, ms, peaks):
+    """The query merge (star_lse_merge over n partials): HBM-bound, n (d + 1) f32 read and a bf16
+    row plus its f32 LSE written per row."""
+    byts = rows * (n * (d + 1) * 4 + 2 * d + 4)
+    sec = ms * 1e-3
+    return {"us": ms * 1e3, "bytes": byts, "gbs": byts / sec / 1e9, "frac_hbm": byts / sec / 1e9 / peaks["hbm_gbs"]}
 
 
 def _ev():
@@ -325,7 +358,7 @@ def run_star(args, rank, world, local_rank):
         raise RuntimeError("device error after warm-up")
 
     K = args.steps
-    evs = [{"p1": _pair(), "p2": _pair(), "dec_span": _tpair()} for _ in range(K)]
+    evs = [{"p1": _pair(), "p2": _pair(), "merge": _tpair(), "dec_span": _tpair()} for _ in range(K)]
     t0, t1 = _ev(), _ev()
     if world > 1:
         dist.barrier()
@@ -347,6 +380,7 @@ def run_star(args, rank, world, local_rank):
 
     p1_ms = statistics.mean(e["p1"][0].elapsed_time(e["p1"][1]) for e in evs)
     p2_ms = statistics.mean(e["p2"][0].elapsed_time(e["p2"][1]) for e in evs)
+    merge_ms = statistics.mean(e["merge"][0].elapsed_time(e["merge"][1]) for e in evs)
     dec_kernel_ms = [ev_dec["dec"][s][0].elapsed_time(ev_dec["dec"][s][1]) for s in range(wl.S)]
     dec_step_ms = statistics.mean(e["dec_span"][0].elapsed_time(e["dec_span"][1]) for e in evs) / wl.S
     flops = wl.phase1_flops()
@@ -366,16 +400,18 @@ def run_star(args, rank, world, local_rank):
         "config": workload_config(wl, world),
         "phase1": {"attn_ms": p1_ms, "ctx_tok_s": wl.context_tokens() / (p1_ms * 1e-3), "tflops": tflops,
                    "frac_bf16_burst": tflops / peaks["bf16"], "frac_bf16_sustained": tflops / peaks["bf16_sustained"]},
-        "phase2": {"attn_ms": p2_ms},
+        "phase2": phase2_roofline(wl, run.shape.n, p2_ms, peaks),
+        "query_merge": merge_roofline(wl.B * wl.T * wl.Hq, run.shape.n, wl.d, merge_ms, peaks),
         "decode": {"us_per_step": 1e3 * dec_step_ms, "kernel_us": 1e3 * statistics.mean(dec_kernel_ms),
                    "bytes_per_step": dec_bytes, "kernel_gbs": dec_gbs, "frac_hbm": dec_gbs / peaks["hbm_gbs"],
                    "step_gbs": dec_bytes / (dec_step_ms * 1e-3) / 1e9,
                    "timing": "us_per_step: the S steps' span in the timed region / S (append, attention, merge "
                              "and launch gaps); kernel_us: the attention kernel alone, one extra untimed step"},
-        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
-                     "frac": tflops / peaks["bf16_sustained"], "traffic": measured_traffic(wl.B, wl.L),
-                     "kernel": f"star_attn_kernel<{wl.d},0> (Phase 1)", "flop_per_launch": flops,
-                     "peak_source": peaks["kind"] + " bf16 sustained"},
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16"], "unit": "TFLOP/s",
+                     "frac": tflops / peaks["bf16"], "traffic": measured_traffic(wl.B, wl.L),
+                     "kernel": f"star_attn_kernel<{wl.d},0> (Phase 1, with its RoPE(Q) pre-pass)",
+                     "flop_per_launch": flops, "peak_source": peaks["kind"] + " bf16 burst",
+                     "peak_sustained": peaks["bf16_sustained"], "frac_sustained": tflops / peaks["bf16_sustained"]},
         "gpu_launches": run.launches_per_step * K,
         "device_status": status,
     }
@@ -485,67 +521,170 @@ def _blas_threads():
         return os.cpu_count() or 1
 
 
-def oracle_phase1_sample(wl, host, blocks, rows_per_block, seed=0):
-    """Time the oracle's Phase-1 rows on a sample: `rows_per_block` rows of each listed block."""
-    import numpy as np
-    import oracle
-    rng = np.random.default_rng(seed)
-    rows = np.concatenate([i * wl.b + rng.choice(wl.b, rows_per_block, replace=False) for i in blocks])
-    rows.sort()
-    k = host["k"].float().numpy().astype(np.float64)
-    v = host["v"].float().numpy().astype(np.float64)
-    q = host["q"][rows].float().numpy().astype(np.float64)
-    pos = host["pos"].numpy().astype(np.int64)
-    apos = host["anchor_pos"].numpy().astype(np.int64) if host.get("anchor_pos") is not None else None
-    t = time.perf_counter()
-    oracle.phase1_rows(rows, q, k, v, pos, wl.b, wl.theta, wl.anchor or None, apos)
-    return len(rows), time.perf_counter() - t
+class OracleSample:
+    """The CPU oracle, as it stands, timed on bounded pieces of one sequence's step.
 
+    Pieces: the roped cache (the context's K through RoPE and the bf16 rounding: the KV
+    append of Phase 1), Phase-1 output rows (``phase1_rows``), the first query tokens'
+    per-block partials plus their merge, and one decode step over the whole cache.  The
+    whole step is extrapolated from their per-unit times, for every sequence of the batch:
+    cache + L_s rows + T query tokens + S decode steps; the work per unit barely changes
+    over a step (decode steps add S << L keys), so the extrapolation is linear.
+    """
 
-def _host_seq0(inp):
-    return {"q": inp["q_ctx"][0].cpu(), "k": inp["k_ctx"][0].cpu(), "v": inp["v_ctx"][0].cpu(),
-            "pos": inp["pos_ctx"][0].cpu(),
-            "anchor_pos": inp["anchor_pos"][0].cpu() if "anchor_pos" in inp else None}
+    def __init__(self, wl, inp, bi=0):
+        import numpy as np
+        self.np, self.wl, self.bi = np, wl, bi
+        f64 = lambda t: t.float().cpu().numpy().astype(np.float64)
+        i64 = lambda t: t.cpu().numpy().astype(np.int64)
+        Ls = wl.ctx_len(bi)
+        self.Ls = Ls
+        self.q_ctx = inp["q_ctx"][bi]                       # rows are converted when sampled
+        self.k, self.v = f64(inp["k_ctx"][bi][:Ls]), f64(inp["v_ctx"][bi][:Ls])
+        self.pos = i64(inp["pos_ctx"][bi][:Ls])
+        self.apos = i64(inp["anchor_pos"][bi]) if "anchor_pos" in inp else None
+        self.qq, self.kq, self.vq = f64(inp["q_query"][bi]), f64(inp["k_query"][bi]), f64(inp["v_query"][bi])
+        self.pos_q = i64(inp["pos_query"][bi])
+        self.qd, self.kd, self.vd = f64(inp["q_dec"][0, bi]), f64(inp["k_dec"][0, bi]), f64(inp["v_dec"][0, bi])
+        self.pos_d = int(inp["pos_dec"][0, bi])
+        self.acc = {"rows": [0.0, 0], "query": [0.0, 0], "decode": [0.0, 0]}
+        self.t_cache = None
+        self.ck = self.ck_full = self.cv_full = None
+
+    def cache(self):
+        import oracle
+        t = time.perf_counter()
+        self.ck = oracle.rope_bf16(self.k, self.pos, self.wl.theta)
+        self.t_cache = time.perf_counter() - t
+        self.ck_full, self.cv_full = oracle.append_tail(self.ck, self.v, self.kq, self.vq, self.pos_q, self.wl.theta)
+
+    def rows(self, blocks, per_block, seed):
+        import oracle
+        np, wl = self.np, self.wl
+        rng = np.random.default_rng(seed)
+        rows = []
+        for i in blocks:
+            lo, hi = i * wl.b, min((i + 1) * wl.b, self.Ls)
+            if hi > lo:
+                rows.append(lo + rng.choice(hi - lo, min(per_block, hi - lo), replace=False))
+        rows = np.sort(np.concatenate(rows))
+        q = self.q_ctx[torch.from_numpy(rows).to(self.q_ctx.device)].float().cpu().numpy().astype(np.float64)
+        t = time.perf_counter()
+        oracle.phase1_rows(rows, q, self.k, self.v, self.pos, wl.b, wl.theta, wl.anchor or None, self.apos)
+        self._add("rows", time.perf_counter() - t, len(rows))
+
+    def query(self, tokens):
+        """The first `tokens` query tokens: their per-block partials over the cache with the tail
+        up to them, and the merge (exactly the work of those tokens)."""
+        import oracle
+        wl, L = self.wl, self.Ls
+        ck, cv = self.ck_full[: L + tokens], self.cv_full[: L + tokens]
+        t = time.perf_counter()
+        Op, Lp = oracle.phase2_partials(self.qq[:tokens], self.pos_q[:tokens], ck, cv, L, wl.b, wl.theta,
+                                        -(-wl.L // wl.b))
+        oracle.lse_merge(Op, Lp)
+        self._add("query", time.perf_counter() - t, tokens)
+
+    def decode(self):
+        import oracle
+        t = time.perf_counter()
+        oracle.decode_step(self.qd, self.kd, self.vd, self.pos_d, self.ck_full, self.cv_full, self.wl.theta)
+        self._add("decode", time.perf_counter() - t, 1)
+
+    def _add(self, key, sec, units):
+        self.acc[key][0] += sec
+        self.acc[key][1] += units
+
+    def per_unit(self, key):
+        sec, units = self.acc[key]
+        return sec / units
+
+    def step_seconds(self):
+        """Extrapolated seconds of one whole step for the batch (every sequence at this one's rates)."""
+        wl = self.wl
+        return sum(self.t_cache * wl.ctx_len(bi) / self.Ls + wl.ctx_len(bi) * self.per_unit("rows")
+                   + wl.T * self.per_unit("query") + wl.S * self.per_unit("decode") for bi in range(wl.B))
+
+    def describe(self):
+        return (f"float64 oracle on sequence {self.bi} of {self.wl.name}: roped cache {self.t_cache:.3g} s; "
+                f"{self.acc['rows'][1]} Phase-1 rows (phase1_rows) at {self.per_unit('rows'):.3g} s/row; "
+                f"{self.acc['query'][1]} query tokens (partials + merge) at {self.per_unit('query'):.3g} s/token; "
+                f"{self.acc['decode'][1]} decode steps at {self.per_unit('decode'):.3g} s/step; value = context "
+                f"tokens / the EXTRAPOLATED whole step ({self.step_seconds():.4g} s = cache + L rows + T query "
+                f"tokens + S decode steps per sequence)")
 
 
 def cpu_baseline(run, rows_per_block):
     wl = run.wl
-    host = _host_seq0(run.inp)
-    nrows, sec = oracle_phase1_sample(wl, host, range(wl.n), rows_per_block)
-    return {"value": nrows / sec, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
-            "sample": f"float64 oracle, Phase-1 output of {nrows} context rows ({rows_per_block} per block, all "
-                      f"{wl.Hq} heads, sequence 0) of {wl.name}; value = rows/s; {sec:.1f} s"}
+    t0 = time.perf_counter()
+    o = OracleSample(wl, run.inp)
+    o.cache()
+    o.rows(range(-(-o.Ls // wl.b)), rows_per_block, seed=0)
+    o.query(min(4, wl.T))
+    o.decode()
+    step = o.step_seconds()
+    return {"value": wl.context_tokens() / step, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+            "sample": o.describe() + f"; sample wall time {time.perf_counter() - t0:.1f} s",
+            "extrapolated_step_s": step}
 
 
 def run_reference(args, rank, world):
+    """The reference arm: the oracle as it stands on the host cores.  Each step is a bounded
+    sample of the workload's step (2 Phase-1 rows of one block, the first query token, one
+    decode step); the value is context tokens per second of the whole step extrapolated from
+    the accumulated per-unit times, the unit and quantity of the CUDA arm."""
     if rank != 0:
         return
     wl = get_config(args.config)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    inp = make_inputs(wl, dev, parts=("ctx",))
-    host = _host_seq0(inp)
+    inp = make_inputs(wl, dev)
+    o = OracleSample(wl, inp)
     del inp
-    rows_per_block = 4
+    o.cache()
+    n_blocks = -(-o.Ls // wl.b)
     W = max(3, args.warmup)
+
+    def one(k, seed):
+        o.rows([k % n_blocks], 2, seed)
+        o.query(1)
+        o.decode()
+
     for w in range(W):
-        oracle_phase1_sample(wl, host, [w % wl.n], rows_per_block, seed=w)
-    tot_rows, tot_sec = 0, 0.0
+        one(w, w)
+    o.acc = {key: [0.0, 0] for key in o.acc}
+    t0 = time.perf_counter()
     for k in range(args.steps):
-        r, s = oracle_phase1_sample(wl, host, [k % wl.n], rows_per_block, seed=100 + k)
-        tot_rows += r
-        tot_sec += s
-    value = tot_rows / tot_sec
+        one(k, 100 + k)
+    sample_s = (time.perf_counter() - t0) / args.steps
+    step = o.step_seconds()
+    value = wl.context_tokens() / step
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": W, "ms_per_step": 1e3 * tot_sec / args.steps, "higher_is_better": True, "scaling": "weak",
+        "warmup": W, "ms_per_step": 1e3 * sample_s, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (same seeded inputs as the CUDA arm)",
         "config": workload_config(wl, world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
-                         "sample": f"each step: float64 oracle Phase-1 output of {rows_per_block} context rows of one "
-                                   f"block (all {wl.Hq} heads) of {wl.name}; value = rows/s"},
+                         "sample": "each step: 2 Phase-1 rows of one block, the first query token's partials and "
+                                   "merge, one decode step; ms_per_step is that sample's time; " + o.describe(),
+                         "extrapolated_step_s": step},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def run_oracle_full(args):
+    """The whole oracle (Phase 1, query partials and merge, every decode step) on the full
+    workload, timed on the host cores; for the small workloads whose full run takes minutes."""
+    import oracle
+    wl = get_config(args.config)
+    inp = make_inputs(wl, "cpu")
+    host = {k: (v.float().numpy().astype("float64") if v.dtype == torch.bfloat16 else v.numpy().astype("int64"))
+            for k, v in inp.items()}
+    t = time.perf_counter()
+    oracle.run_star(host, wl.L, wl.b, wl.theta, anchor=wl.anchor or None)
+    sec = time.perf_counter() - t
+    print(json.dumps({"oracle_full": wl.name, "seconds": sec, "ctx_tok_s": wl.context_tokens() / sec,
+                      "cores": _blas_threads(), "nproc": os.cpu_count()}), flush=True)
 
 
 def run_layers(args):
@@ -621,6 +760,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.oracle_full:
+        run_oracle_full(args)
         return
     if args.layers > 0:
         run_layers(args)

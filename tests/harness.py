@@ -8,6 +8,7 @@ with the stated tolerances.
 from __future__ import annotations
 
 import dataclasses
+import os
 
 import numpy as np
 import torch
@@ -19,6 +20,10 @@ from synth import Workload, make_inputs
 MAX_ABS = 1.5e-2
 MEAN_ABS = 2e-3
 LSE_ABS = 1e-3
+
+# Every assert_out call: (test id, what, elements over MAX_ABS that the |O| >= 4 bound
+# admitted, elements compared).  The conftest prints the totals per test.
+ALLOWANCE: list[tuple[str, str, int, int]] = []
 
 
 def shape_of(wl: Workload) -> star.StarShape:
@@ -119,6 +124,8 @@ def assert_out(gpu, ref, what: str):
     assert np.all(np.isfinite(g)), f"{what}: non-finite output"
     bound = np.maximum(MAX_ABS, 0.5 * bf16_spacing(r) + 4e-3)
     over = np.abs(g - r) > bound
+    relaxed = int(((np.abs(g - r) > MAX_ABS) & ~over).sum())
+    ALLOWANCE.append((os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0], what, relaxed, int(r.size)))
     worst = np.unravel_index(np.argmax(np.abs(g - r) - bound), r.shape) if r.size else None
     assert not over.any() and e.mean_abs <= MEAN_ABS, (
         f"{what}: max abs {e.max_abs:.3e}, mean abs {e.mean_abs:.3e} (<= {MEAN_ABS}); "

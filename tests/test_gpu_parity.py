@@ -170,7 +170,20 @@ def test_invalid_arguments_launch_nothing():
     assert star.star_device_status() == 0
 
 
-def _large_check(wl: Workload, rows_per_block: int, dec_steps_checked):
+def _decode_reference(inp, bi, ck, cv, theta):
+    """Every decode step of sequence bi at once: the step-s token, roped at its position,
+    attends to the cache [context, query tail, decode tokens 0..s] (oracle.global_attention
+    with the rows' cache indices; the pins show the S chained decode steps equal it)."""
+    h = H()
+    S = inp["q_dec"].shape[0]
+    dpos = inp["pos_dec"][:, bi].cpu().numpy().astype(np.int64)
+    qd = oracle.rope_bf16(h.to64(inp["q_dec"][:, bi, 0]), dpos, theta)
+    ck, cv = oracle.append_tail(ck, cv, h.to64(inp["k_dec"][:, bi, 0]), h.to64(inp["v_dec"][:, bi, 0]), dpos, theta)
+    rows = ck.shape[0] - S + np.arange(S)
+    return oracle.global_attention(qd, rows, ck, cv)
+
+
+def _large_check(wl: Workload, rows_per_block: int):
     h = H()
     inp = make_inputs(wl, "cuda")
     res = h.run_gpu(wl, inp)
@@ -194,49 +207,45 @@ def _large_check(wl: Workload, rows_per_block: int, dec_steps_checked):
         h.assert_lse(res["lse_part"][:, bi], Lp, "phase2 partial LSE")
         h.assert_out(res["o_query"][bi], Oq, "merged O")
         h.assert_lse(res["lse_query"][bi], Lq, "merged LSE")
-        for s in range(wl.S):
-            kd, vd = h.to64(inp["k_dec"][s, bi]), h.to64(inp["v_dec"][s, bi])
-            p = int(inp["pos_dec"][s, bi])
-            if s in dec_steps_checked:
-                O, LSE, ck, cv = oracle.decode_step(h.to64(inp["q_dec"][s, bi]), kd, vd, p, ck, cv, theta)
-                h.assert_out(res["o_dec"][s, bi], O, f"decode step {s} O")
-                h.assert_lse(res["lse_dec"][s, bi], LSE[0], f"decode step {s} LSE")
-            else:
-                ck, cv = oracle.append_tail(ck, cv, kd, vd, [p], theta)
+        # Every decode step.
+        Od, Ld = _decode_reference(inp, bi, ck, cv, theta)
+        h.assert_out(res["o_dec"][:, bi, 0], Od, "decode O (every step)")
+        h.assert_lse(res["lse_dec"][:, bi], Ld, "decode LSE (every step)")
 
 
 def test_llama8b_32k_sampled_rows_and_full_merge():
     wl = get_config("llama8b-32k")
-    _large_check(wl, 60, set(range(wl.S)))
+    _large_check(wl, 60)
 
 
 def test_llama8b_128k_b32768_sampled_rows_and_full_merge():
     wl = get_config("llama8b-128k-b32768")
-    _large_check(wl, 28, {0, 1, wl.S - 1})
+    _large_check(wl, 28)
 
 
 @pytest.mark.parametrize("b", [4096, 8192, 16384])
 def test_llama8b_128k_block_sweep_sampled(b):
     wl = get_config(f"llama8b-128k-b{b}")
-    _large_check(wl, 6, {0, wl.S - 1})
+    _large_check(wl, 6)
 
 
 def test_llama70b_128k_sampled():
     """B = 2 sequences, GQA group 8, 128 query tokens (one full query tile per head)."""
     wl = get_config("llama70b-128k")
-    _large_check(wl, 6, {0, wl.S - 1})
+    _large_check(wl, 6)
 
 
 def test_million_token_context_sampled_streaming_oracle():
     """1M context (8 blocks of 131072): sampled Phase-1 rows, every Phase-2 partial,
-    the merged query output and the first decode step, with the oracle run block by
-    block (its partials merged by oracle.lse_merge) so host memory stays small."""
+    the merged query output and every decode step, with the oracle run block by block
+    (its per-block partials merged by oracle.lse_merge, exact by the merge pins) so
+    host memory stays small."""
     h = H()
     wl = get_config("ctx-1m")
     inp = make_inputs(wl, "cuda")
-    res = h.run_gpu(wl, inp, phases=("phase1", "phase2"))
+    res = h.run_gpu(wl, inp)
     assert res["status"] == 0
-    theta, b, L = wl.theta, wl.b, wl.L
+    theta, b, L, T, S = wl.theta, wl.b, wl.L, wl.T, wl.S
     k = h.to64(inp["k_ctx"][0])
     v = h.to64(inp["v_ctx"][0])
     pos = inp["pos_ctx"][0].cpu().numpy().astype(np.int64)
@@ -248,48 +257,32 @@ def test_million_token_context_sampled_streaming_oracle():
     qr = oracle.rope_bf16(h.to64(inp["q_query"][0]), qpos, theta)
     kq = oracle.rope_bf16(h.to64(inp["k_query"][0]), qpos, theta)
     vq = h.to64(inp["v_query"][0])
-    row_idx = L + np.arange(wl.T)
-    Op, Lp = [], []
+    dpos = inp["pos_dec"][:, 0].cpu().numpy().astype(np.int64)
+    qd = oracle.rope_bf16(h.to64(inp["q_dec"][:, 0, 0]), dpos, theta)
+    kd = oracle.rope_bf16(h.to64(inp["k_dec"][:, 0, 0]), dpos, theta)
+    vd = h.to64(inp["v_dec"][:, 0, 0])
+    q_idx = L + np.arange(T)
+    d_idx = L + T + np.arange(S)
+    Op, Lp, Od, Ld = [], [], [], []
     for i in range(wl.n):
         ck = oracle.rope_bf16(k[i * b:(i + 1) * b], pos[i * b:(i + 1) * b], theta)
         cv = v[i * b:(i + 1) * b]
         key_idx = np.arange(i * b, (i + 1) * b)
-        if i == wl.n - 1:
-            ck, cv = np.concatenate([ck, kq]), np.concatenate([cv, vq])
-            key_idx = np.concatenate([key_idx, row_idx])
-        O, LS = oracle.attend(qr, ck, cv, key_idx[None, :] <= row_idx[:, None])
+        if i == wl.n - 1:                      # the tail: query tokens, then the decode tokens
+            ck, cv = np.concatenate([ck, kq, kd]), np.concatenate([cv, vq, vd])
+            key_idx = np.concatenate([key_idx, q_idx, d_idx])
+        O, LS = oracle.attend(qr, ck, cv, key_idx[None, :] <= q_idx[:, None])
         Op.append(O)
         Lp.append(LS)
+        O, LS = oracle.attend(qd, ck, cv, key_idx[None, :] <= d_idx[:, None])
+        Od.append(O)
+        Ld.append(LS)
     Op, Lp = np.stack(Op), np.stack(Lp)
     h.assert_out(res["o_part"][:, 0], Op, "1M phase2 partial O")
     h.assert_lse(res["lse_part"][:, 0], Lp, "1M phase2 partial LSE")
     Oq, Lq = oracle.lse_merge(Op, Lp)
     h.assert_out(res["o_query"][0], Oq, "1M merged O")
     h.assert_lse(res["lse_query"][0], Lq, "1M merged LSE")
-    # First decode step: GPU through the C ABI; oracle as per-block partials + merge.
-    import block_sparse_attention_star_b200 as star
-    shape, cache = res["shape"], res["cache"]
-    ws = star.workspace(shape, star.STAR_OP_DECODE)
-    o_dec = torch.empty((1, 1, wl.Hq, wl.d), dtype=torch.bfloat16, device="cuda")
-    l_dec = torch.empty((1, wl.Hq), dtype=torch.float32, device="cuda")
-    cur = L + wl.T
-    star.star_decode_step(shape, cache, inp["q_dec"][0], inp["k_dec"][0], inp["v_dec"][0], inp["pos_dec"][0], cur,
-                          o_dec, l_dec, ws)
-    torch.cuda.synchronize()
-    assert star.star_device_status() == 0
-    dpos = int(inp["pos_dec"][0, 0])
-    qd = oracle.rope_bf16(h.to64(inp["q_dec"][0, 0]), [dpos], theta)
-    kd = oracle.rope_bf16(h.to64(inp["k_dec"][0, 0]), [dpos], theta)
-    vd = h.to64(inp["v_dec"][0, 0])
-    Od, Ld = [], []
-    for i in range(wl.n):
-        ck = oracle.rope_bf16(k[i * b:(i + 1) * b], pos[i * b:(i + 1) * b], theta)
-        cv = v[i * b:(i + 1) * b]
-        if i == wl.n - 1:
-            ck, cv = np.concatenate([ck, kq, kd]), np.concatenate([cv, vq, vd])
-        O, LS = oracle.attend(qd, ck, cv)
-        Od.append(O)
-        Ld.append(LS)
     Odm, Ldm = oracle.lse_merge(np.stack(Od), np.stack(Ld))
-    h.assert_out(o_dec[0], Odm, "1M decode O")
-    h.assert_lse(l_dec[0], Ldm[0], "1M decode LSE")
+    h.assert_out(res["o_dec"][:, 0, 0], Odm, "1M decode O (every step)")
+    h.assert_lse(res["lse_dec"][:, 0], Ldm, "1M decode LSE (every step)")
