@@ -55,6 +55,9 @@ def parse_args():
     ap.add_argument("--cpu-rows", type=int, default=8, help="Phase-1 rows per block in the oracle sample")
     ap.add_argument("--oracle-full", action="store_true",
                     help="time the whole CPU oracle on the full workload (small workloads only) and exit")
+    ap.add_argument("--shard", action="store_true",
+                    help="multi-GPU Star Attention: every rank owns a block range of the same sequences "
+                         "(Phase 1 on its blocks, Phase-2 and decode partials exchanged and merged)")
     ap.add_argument("--layers", type=int, default=0,
                     help="time N layers of context encoding (star_encode_layers, random projections) instead")
     return ap.parse_args()
@@ -235,6 +238,102 @@ class StarRun:
             ev["dec_span"][1].record()
         if ev:
             s.star_set_trace_events(None, None)
+
+
+class ShardRun:
+    """One rank's share of a workload when the context's blocks are sharded over the ranks:
+    its block range of every sequence (the same sequences on every rank), the anchor's
+    tokens when the range does not hold block 1, and the tail on the rank with the last block."""
+
+    def __init__(self, wl, device):
+        import block_sparse_attention_star_b200 as star
+        from block_sparse_attention_star_b200.shard import ShardExchange
+        self.star, self.wl, self.dev = star, wl, device
+        inp = make_inputs(wl, device)
+        self.shape = workload_shape(wl)
+        self.ex = ShardExchange(wl.n, device=device)
+        i0, i1 = self.ex.begin, self.ex.end
+        self.tail = i1 == wl.n
+        sl = slice(i0 * wl.b, i1 * wl.b)
+        a = wl.a
+        self.ctx = {x: inp[x][:, sl].contiguous() for x in ("q_ctx", "k_ctx", "v_ctx", "pos_ctx")}
+        self.anchor = {x: inp[x][:, :a].contiguous() for x in ("k_ctx", "v_ctx", "pos_ctx")}
+        self.query = {x: inp[x] for x in ("q_query", "k_query", "v_query", "pos_query")}
+        self.dec = {x: inp[x] for x in ("q_dec", "k_dec", "v_dec", "pos_dec")}
+        del inp
+        self.cache = star.PagedKVCache(self.shape, device=device)
+        self.o_ctx = torch.empty_like(self.ctx["q_ctx"])
+        nl = i1 - i0
+        self.o_part = torch.empty((nl, wl.B, wl.T, wl.Hq, wl.d), dtype=torch.float32, device=device)
+        self.lse_part = torch.empty((nl, wl.B, wl.T, wl.Hq), dtype=torch.float32, device=device)
+        self.ws2 = star.workspace(self.shape, star.STAR_OP_PHASE2, wl.T, device)
+        self.wsd = star.workspace(self.shape, star.STAR_OP_DECODE, 0, device)
+        self.o_q = torch.empty((wl.B, wl.T, wl.Hq, wl.d), dtype=torch.bfloat16, device=device)
+        self.lse_q = torch.empty((wl.B, wl.T, wl.Hq), dtype=torch.float32, device=device)
+        self.po = torch.empty((1, wl.B, wl.Hq, wl.d), dtype=torch.float32, device=device)
+        self.pl = torch.empty((1, wl.B, wl.Hq), dtype=torch.float32, device=device)
+        self.o_dec = torch.empty((wl.S, wl.B, wl.Hq, wl.d), dtype=torch.bfloat16, device=device)
+        self.lse_dec = torch.empty((wl.S, wl.B, wl.Hq), dtype=torch.float32, device=device)
+
+    def step(self):
+        s, wl, c, sh = self.star, self.wl, self.ctx, self.ex.shard()
+        s.star_phase1_encode_shard(self.shape, self.cache, sh, c["q_ctx"], c["k_ctx"], c["v_ctx"], c["pos_ctx"],
+                                   self.anchor["k_ctx"], self.anchor["v_ctx"], self.anchor["pos_ctx"], self.o_ctx)
+        q = self.query
+        s.star_phase2_partial_shard(self.shape, self.cache, sh, q["q_query"], q["k_query"] if self.tail else None,
+                                    q["v_query"] if self.tail else None, q["pos_query"], wl.T, self.o_part,
+                                    self.lse_part, self.ws2)
+        rows = wl.B * wl.T * wl.Hq
+        self.ex.gather_merge(self.o_part.view(-1, rows, wl.d), self.lse_part.view(-1, rows), self.o_q, self.lse_q)
+        d = self.dec
+        for st in range(wl.S):
+            s.star_decode_partial_shard(self.shape, self.cache, sh, d["q_dec"][st], d["k_dec"][st], d["v_dec"][st],
+                                        d["pos_dec"][st], wl.L + wl.T + st, self.po[0], self.pl[0], self.wsd)
+            self.ex.gather_merge(self.po.view(1, -1, wl.d), self.pl.view(1, -1), self.o_dec[st], self.lse_dec[st],
+                                 slots=1)
+
+
+def run_shard(args, rank, world, local_rank):
+    """Blocks sharded over the ranks: the whole job processes one batch of sequences per step
+    (strong scaling: the total work is fixed as the rank count grows)."""
+    import torch.distributed as dist
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = get_config(args.config)
+    run = ShardRun(wl, dev)
+    for _ in range(max(3, args.warmup)):
+        run.step()
+    torch.cuda.synchronize()
+    if run.star.star_device_status() != 0:
+        raise RuntimeError("device error after warm-up")
+    K = args.steps
+    t0, t1 = _ev(), _ev()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        t0.record()
+        for _ in range(K):
+            run.step()
+        t1.record()
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    status = run.star.star_device_status()
+    ms_step = max_over_ranks(t0.elapsed_time(t1), dev) / K
+    if rank == 0:
+        nl = run.ex.n_local
+        line = {
+            "metric": METRIC, "value": wl.context_tokens() / (ms_step * 1e-3), "unit": UNIT, "n_gpus": world,
+            "steps": K, "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) bf16; 1% of context key rows x8 where the workload says peaky)",
+            "config": dict(workload_config(wl, world), parallelism=f"context blocks sharded over {world} GPUs"),
+            "exchange": f"per query call and per decode step: all-gather of the f32 (O, LSE) partials "
+                        f"(rank 0 holds {nl} of {wl.n} blocks), then star_lse_merge on every rank",
+            "device_status": status, "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
 
 
 def measured_traffic(B: int, L: int):
@@ -773,7 +872,10 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     try:
-        run_star(args, rank, world, local_rank)
+        if args.shard:
+            run_shard(args, rank, world, local_rank)
+        else:
+            run_star(args, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

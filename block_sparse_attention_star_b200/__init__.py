@@ -72,6 +72,11 @@ class StarShape(ctypes.Structure):
         return sh
 
 
+class StarShard(ctypes.Structure):
+    """Blocks [block_begin, block_end) of every sequence, owned by one GPU (star.h star_shard)."""
+    _fields_ = [("block_begin", ctypes.c_int32), ("block_end", ctypes.c_int32)]
+
+
 class StarCache(ctypes.Structure):
     _fields_ = [
         ("k_pool", ctypes.c_void_p), ("v_pool", ctypes.c_void_p), ("page_table", ctypes.c_void_p),
@@ -112,6 +117,12 @@ def lib() -> ctypes.CDLL:
             "star_decode_step_noalloc": ([P(StarShape), P(StarCache), V, V, V, V, I32, V, V, V], ctypes.c_int),
             "star_encode_layers": ([P(StarShape), I32, P(StarCache), V, V, V, V, V, V, LAYER_FN, V, V], ctypes.c_int),
             "star_debug_set": ([ctypes.c_uint64, I32], ctypes.c_int),
+            "star_phase1_encode_shard": ([P(StarShape), P(StarCache), P(StarShard), V, V, V, V, V, V, V, V, V],
+                                         ctypes.c_int),
+            "star_phase2_partial_shard": ([P(StarShape), P(StarCache), P(StarShard), V, V, V, V, I32, V, V, V, SZ, V],
+                                          ctypes.c_int),
+            "star_decode_partial_shard": ([P(StarShape), P(StarCache), P(StarShard), V, V, V, V, I32, V, V, V, SZ, V],
+                                          ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -311,6 +322,37 @@ def star_device_status(stream=None) -> int:
     rc = lib().star_device_status(_stream(stream), ctypes.byref(code))
     _check(rc)
     return code.value
+
+
+def star_phase1_encode_shard(shape, cache: PagedKVCache, shard: StarShard, q, k, v, pos, k_anchor, v_anchor,
+                             pos_anchor, out, stream=None):
+    _check(lib().star_phase1_encode_shard(ctypes.byref(shape), ctypes.byref(cache.c), ctypes.byref(shard),
+                                          _ptr(q, "q", torch.bfloat16), _ptr(k, "k", torch.bfloat16),
+                                          _ptr(v, "v", torch.bfloat16), _ptr(pos, "pos", torch.int32),
+                                          _ptr(k_anchor, "k_anchor", torch.bfloat16),
+                                          _ptr(v_anchor, "v_anchor", torch.bfloat16),
+                                          _ptr(pos_anchor, "pos_anchor", torch.int32),
+                                          _ptr(out, "out", torch.bfloat16), _stream(stream)))
+
+
+def star_phase2_partial_shard(shape, cache: PagedKVCache, shard: StarShard, q, k, v, q_pos, T: int, o_part, lse_part,
+                              ws, stream=None):
+    _check(lib().star_phase2_partial_shard(ctypes.byref(shape), ctypes.byref(cache.c), ctypes.byref(shard),
+                                           _ptr(q, "q", torch.bfloat16), _ptr(k, "k", torch.bfloat16),
+                                           _ptr(v, "v", torch.bfloat16), _ptr(q_pos, "q_pos", torch.int32), T,
+                                           _ptr(o_part, "o_part", torch.float32),
+                                           _ptr(lse_part, "lse_part", torch.float32), _ptr(ws, "ws"),
+                                           ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def star_decode_partial_shard(shape, cache: PagedKVCache, shard: StarShard, q, k, v, pos, cur_len: int, o_part,
+                              lse_part, ws, stream=None):
+    _check(lib().star_decode_partial_shard(ctypes.byref(shape), ctypes.byref(cache.c), ctypes.byref(shard),
+                                           _ptr(q, "q", torch.bfloat16), _ptr(k, "k", torch.bfloat16),
+                                           _ptr(v, "v", torch.bfloat16), _ptr(pos, "pos", torch.int32), cur_len,
+                                           _ptr(o_part, "o_part", torch.float32),
+                                           _ptr(lse_part, "lse_part", torch.float32), _ptr(ws, "ws"),
+                                           ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def star_debug_set(wait_limit_ns: int = 0, flags: int = 0) -> None:

@@ -149,6 +149,25 @@ int phase2_chunks_per_block(const star_shape* s, int T) {
   return best;
 }
 
+// The same choice for a shard of nblk blocks, capped so that its chunk partials never
+// outnumber the whole context's (the Phase-2 workspace is sized for those).
+int phase2_chunks_per_block_shard(const star_shape* s, int T, int nblk) {
+  const int G = s->Hq / s->Hkv;
+  int TQ = 1;
+  while (TQ < T && TQ < 128) TQ <<= 1;
+  const int HT = 128 / TQ;
+  const int NTT = (T + TQ - 1) / TQ;
+  const int NHT = (G + HT - 1) / HT;
+  const int npairs = (NTT * NHT + 1) / 2;
+  const int64_t base = (int64_t)nblk * s->B * s->Hkv * npairs;
+  const int64_t max_parts = (int64_t)s->n * phase2_chunks_per_block(s, T);
+  const int nb = s->b / 128;
+  int best = 1;
+  for (int c = 1; c <= nb; ++c)
+    if (nb % c == 0 && base * c <= num_sms() && (int64_t)nblk * c <= max_parts) best = c;
+  return best;
+}
+
 // Phase-2 scratch: RoPE(q) (bf16 [B][T][Hq][d]), then, when blocks are split into
 // chunks, the chunk partials (f32 O, then LSE).
 size_t phase2_q_bytes(const star_shape* s, int T) { return round_up((size_t)s->B * T * s->Hq * s->d * 2, 256); }
@@ -507,6 +526,8 @@ int star_decode_step(const star_shape* shape, const star_cache* cache, const voi
   a.v_new = v;
   a.pos = pos;
   a.n_keys = n_keys;
+  a.k_lo = 0;
+  a.append = 1;
   a.shift = shift_of(shape);
   a.chunk = chunk;
   a.cache = cv;
@@ -520,6 +541,211 @@ int star_decode_step(const star_shape* shape, const star_cache* cache, const voi
   if (e != cudaSuccess) return cuda_fail(e, "decode attention launch");
   e = star::launch_lse_merge(1, nch, (int64_t)rows, shape->d, a.o_ws, a.lse_ws, out, true, lse_out, st);
   return e == cudaSuccess ? STAR_OK : cuda_fail(e, "decode merge launch");
+}
+
+// ---------------------------------------------------------------------------
+// Shards: a contiguous block range per GPU
+// ---------------------------------------------------------------------------
+static int check_shard(const star_shape* s, const star_shard* sh) {
+  if (!sh) return fail(STAR_ERR_INVALID_ARG, "shard is NULL");
+  if (sh->block_begin < 0 || sh->block_end <= sh->block_begin || sh->block_end > s->n)
+    return fail(STAR_ERR_INVALID_ARG, "shard blocks [%d, %d) outside [0, n = %d)", sh->block_begin, sh->block_end, s->n);
+  if (s->seq_len) return fail(STAR_ERR_UNSUPPORTED_SHAPE, "shards need sequences of one length (seq_len must be NULL)");
+  return STAR_OK;
+}
+
+int star_phase1_encode_shard(const star_shape* shape, const star_cache* cache, const star_shard* shard, const void* q,
+                             const void* k, const void* v, const int32_t* pos, const void* k_anchor,
+                             const void* v_anchor, const int32_t* pos_anchor, void* out, star_stream_t stream) {
+  int rc = check_shape(shape);
+  if (!rc) rc = check_cache(shape, cache);
+  if (!rc) rc = check_shard(shape, shard);
+  if (rc) return rc;
+  STAR_REQUIRE_PTR(q, "q");
+  STAR_REQUIRE_PTR(k, "k");
+  STAR_REQUIRE_PTR(v, "v");
+  STAR_REQUIRE_PTR4(pos, "pos");
+  STAR_REQUIRE_PTR(out, "out");
+  const int i0 = shard->block_begin, nblk = shard->block_end - shard->block_begin;
+  const int anchor = anchor_of(shape);
+  if (i0 > 0) {
+    STAR_REQUIRE_PTR(k_anchor, "k_anchor");
+    STAR_REQUIRE_PTR(v_anchor, "v_anchor");
+    STAR_REQUIRE_PTR4(pos_anchor, "pos_anchor");
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  const star::CacheView cv = view(shape, cache);
+  const star::RopeTable rt = rope_table(shape);
+  // The range's own tokens at their cache slots, and the anchor (block 1's first a tokens,
+  // read by every later block) when the range does not hold block 1.
+  cudaError_t e = star::launch_rope_append(k, v, pos, shape->B, nblk * shape->b, i0 * shape->b, shape->Hkv, shape->d,
+                                           cv, rt, st);
+  if (e == cudaSuccess && i0 > 0)
+    e = star::launch_rope_append(k_anchor, v_anchor, pos_anchor, shape->B, anchor, 0, shape->Hkv, shape->d, cv, rt, st);
+  if (e == cudaSuccess && shard->block_end == shape->n)
+    e = star::launch_zero_slots(shape->B, shape->L, shape->L + (int)round_up(shape->T_max, 128), shape->Hkv, shape->d,
+                                cv, st);
+  if (e != cudaSuccess) return cuda_fail(e, "phase1 shard kv append");
+  star::AttnLaunch a;
+  memset(&a, 0, sizeof(a));
+  a.mode = 0;
+  a.anchor = anchor;
+  a.B = shape->B;
+  a.Hq = shape->Hq;
+  a.Hkv = shape->Hkv;
+  a.d = shape->d;
+  a.L = shape->L;
+  a.b = shape->b;
+  a.n = shape->n;
+  a.q = out;
+  a.Ntok = shape->L;
+  a.cache = cv;
+  a.out_bf16 = out;
+  a.chunks_per_block = 1;
+  a.scale_log2 = scale_log2(shape);
+  a.blk0 = i0;
+  a.nblk = nblk;
+  const char* why = nullptr;
+  trace_begin(st);
+  e = star::launch_rope_q(q, pos, shape->B, nblk * shape->b, shape->Hq, shape->d, out, rt, st);
+  if (e == cudaSuccess) e = star::launch_attention(a, st, &why);
+  trace_end(st);
+  if (e != cudaSuccess) return why ? fail(STAR_ERR_CUDA, "%s", why) : cuda_fail(e, "phase1 shard attention launch");
+  return STAR_OK;
+}
+
+int star_phase2_partial_shard(const star_shape* shape, const star_cache* cache, const star_shard* shard, const void* q,
+                              const void* k, const void* v, const int32_t* q_pos, int32_t T, float* o_part,
+                              float* lse_part, void* ws, size_t ws_bytes, star_stream_t stream) {
+  int rc = check_shape(shape);
+  if (!rc) rc = check_cache(shape, cache);
+  if (!rc) rc = check_shard(shape, shard);
+  if (rc) return rc;
+  STAR_REQUIRE_PTR(q, "q");
+  STAR_REQUIRE_PTR4(q_pos, "q_pos");
+  STAR_REQUIRE_PTR(o_part, "o_part");
+  STAR_REQUIRE_PTR4(lse_part, "lse_part");
+  if ((k == nullptr) != (v == nullptr)) return fail(STAR_ERR_INVALID_ARG, "k and v must both be given or both be NULL");
+  if (T <= 0 || T > shape->T_max) return fail(STAR_ERR_INVALID_ARG, "T (%d) must be in [1, T_max=%d]", T, shape->T_max);
+  const bool tail = shard->block_end == shape->n;
+  if (k && !tail) return fail(STAR_ERR_INVALID_ARG, "only the shard holding the last block appends the query's k, v");
+  const size_t need = phase2_ws_bytes(shape, T);
+  STAR_REQUIRE_PTR(ws, "ws");
+  if (ws_bytes < need) return fail(STAR_ERR_CAPACITY, "workspace %zu bytes < %zu needed", ws_bytes, need);
+  cudaStream_t st = (cudaStream_t)stream;
+  const star::CacheView cv = view(shape, cache);
+  const star::RopeTable rt = rope_table(shape);
+  if (k) {
+    STAR_REQUIRE_PTR(k, "k");
+    STAR_REQUIRE_PTR(v, "v");
+    cudaError_t e = star::launch_rope_append(k, v, q_pos, shape->B, T, shape->L, shape->Hkv, shape->d, cv, rt, st);
+    if (e != cudaSuccess) return cuda_fail(e, "phase2 shard kv append");
+  }
+  const int nblk = shard->block_end - shard->block_begin;
+  const int cpb = phase2_chunks_per_block_shard(shape, T, nblk);
+  const size_t rows = (size_t)shape->B * T * shape->Hq;
+  const size_t parts = (size_t)nblk * cpb;
+  void* q_rot = ws;
+  char* chunk_ws = reinterpret_cast<char*>(ws) + phase2_q_bytes(shape, T);
+  float* o_dst = o_part;
+  float* l_dst = lse_part;
+  if (cpb > 1) {
+    o_dst = reinterpret_cast<float*>(chunk_ws);
+    l_dst = reinterpret_cast<float*>(chunk_ws + round_up(parts * rows * shape->d * sizeof(float), 256));
+  }
+  star::AttnLaunch a;
+  memset(&a, 0, sizeof(a));
+  a.mode = 1;
+  a.B = shape->B;
+  a.Hq = shape->Hq;
+  a.Hkv = shape->Hkv;
+  a.d = shape->d;
+  a.L = shape->L;
+  a.b = shape->b;
+  a.n = shape->n;
+  a.q = q_rot;
+  a.Ntok = T;
+  a.cache = cv;
+  a.out_f32 = o_dst;
+  a.lse_f32 = l_dst;
+  a.chunks_per_block = cpb;
+  a.scale_log2 = scale_log2(shape);
+  a.blk0 = shard->block_begin;
+  a.nblk = nblk;
+  a.no_tail = tail ? 0 : 1;
+  const char* why = nullptr;
+  trace_begin(st);
+  cudaError_t e = star::launch_rope_q(q, q_pos, shape->B, T, shape->Hq, shape->d, q_rot, rt, st);
+  if (e == cudaSuccess) e = star::launch_attention(a, st, &why);
+  trace_end(st);
+  if (e != cudaSuccess) return why ? fail(STAR_ERR_CUDA, "%s", why) : cuda_fail(e, "phase2 shard attention launch");
+  if (cpb > 1) {
+    e = star::launch_lse_merge(nblk, cpb, (int64_t)rows, shape->d, o_dst, l_dst, o_part, false, lse_part, st);
+    if (e != cudaSuccess) return cuda_fail(e, "phase2 shard chunk merge");
+  }
+  return STAR_OK;
+}
+
+int star_decode_partial_shard(const star_shape* shape, const star_cache* cache, const star_shard* shard, const void* q,
+                              const void* k, const void* v, const int32_t* pos, int32_t cur_len, float* o_part,
+                              float* lse_part, void* ws, size_t ws_bytes, star_stream_t stream) {
+  int rc = check_shape(shape);
+  if (!rc) rc = check_cache(shape, cache);
+  if (!rc) rc = check_shard(shape, shard);
+  if (rc) return rc;
+  STAR_REQUIRE_PTR(q, "q");
+  STAR_REQUIRE_PTR4(o_part, "o_part");
+  STAR_REQUIRE_PTR4(lse_part, "lse_part");
+  STAR_REQUIRE_PTR(ws, "ws");
+  const bool tail = shard->block_end == shape->n;
+  if (tail) {
+    STAR_REQUIRE_PTR(k, "k");
+    STAR_REQUIRE_PTR(v, "v");
+    STAR_REQUIRE_PTR4(pos, "pos");
+    if (cur_len < shape->L || cur_len >= shape->L + shape->T_max)
+      return fail(STAR_ERR_CAPACITY, "cur_len %d outside [L = %d, L + T_max = %d)", cur_len, shape->L,
+                  shape->L + shape->T_max);
+  } else {
+    STAR_REQUIRE_PTR4(pos, "pos");
+  }
+  const size_t need = decode_ws_bytes(shape);
+  if (ws_bytes < need) return fail(STAR_ERR_CAPACITY, "workspace %zu bytes < %zu needed", ws_bytes, need);
+  cudaStream_t st = (cudaStream_t)stream;
+  // Keys of the range: its blocks' context keys, plus the tail up to the new token (appended
+  // here) on the shard that holds the last block.
+  const int k_lo = shard->block_begin * shape->b;
+  const int n_keys = tail ? cur_len + 1 : shard->block_end * shape->b;
+  const int chunk_cap = decode_chunk(shape);
+  const size_t nch_max = (size_t)star::decode_num_chunks(shape->L + shape->T_max, chunk_cap);
+  int chunk = star::decode_pick_chunk(shape->B, shape->Hkv, shape->Hq / shape->Hkv, n_keys - k_lo, num_sms());
+  while ((size_t)star::decode_num_chunks(n_keys - k_lo, chunk) > nch_max) chunk += 128;  // fits the workspace
+  const int nch = star::decode_num_chunks(n_keys - k_lo, chunk);
+  const size_t rows = (size_t)shape->B * shape->Hq;
+  star::DecodeLaunch a;
+  memset(&a, 0, sizeof(a));
+  a.B = shape->B;
+  a.Hq = shape->Hq;
+  a.Hkv = shape->Hkv;
+  a.d = shape->d;
+  a.q = q;
+  a.k_new = tail ? k : q;  // read only by the CTA that appends (tail shard)
+  a.v_new = tail ? v : q;
+  a.pos = pos;
+  a.n_keys = n_keys;
+  a.k_lo = k_lo;
+  a.append = tail ? 1 : 0;
+  a.chunk = chunk;
+  a.cache = view(shape, cache);
+  a.o_ws = reinterpret_cast<float*>(ws);
+  a.lse_ws = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + round_up(nch_max * rows * shape->d * sizeof(float), 256));
+  a.scale_log2 = scale_log2(shape);
+  a.rope = rope_table(shape);
+  trace_begin(st);
+  cudaError_t e = star::launch_decode(a, st);
+  trace_end(st);
+  if (e != cudaSuccess) return cuda_fail(e, "decode shard launch");
+  e = star::launch_lse_merge(1, nch, (int64_t)rows, shape->d, a.o_ws, a.lse_ws, o_part, false, lse_part, st);
+  return e == cudaSuccess ? STAR_OK : cuda_fail(e, "decode shard merge launch");
 }
 
 int star_set_trace_events(void* start_event, void* stop_event) {

@@ -66,6 +66,8 @@ struct DecParams {
   float* lse_ws;       // [nchunks][B*Hq]
   int max_pages, num_pages, P;
   int B, Hq, Hkv, n_keys, chunk, nchunks;
+  int k_lo;                  // first key of the range (0, or a shard's first block's first key)
+  int append;                // the range holds the new token's slot n_keys - 1 (it is appended here)
   int item_base, num_items;  // this launch: items [item_base, num_items)
   float scale_log2;
   SeqShift sh;               // sequence bi has n_keys + delta[bi] keys (sh.on = 0: all n_keys)
@@ -138,11 +140,11 @@ __device__ __forceinline__ DecItem dec_item(const DecParams& p, int idx) {
     it.c = p.nchunks - ne + (w - it.g * ne);
   }
   it.n_keys = p.n_keys + (p.sh.on ? p.sh.delta[it.bi] : 0);
-  it.k_begin = it.c * p.chunk;
+  it.k_begin = p.k_lo + it.c * p.chunk;
   it.k_end = min(it.k_begin + p.chunk, it.n_keys);
   // A chunk past a shorter sequence's keys is empty (0 tiles): its partial is O = 0, LSE = -inf.
   it.ntiles = it.k_end > it.k_begin ? (it.k_end - it.k_begin + kTileKeys - 1) / kTileKeys : 0;
-  it.last = (it.c == (it.n_keys - 1) / p.chunk);
+  it.last = p.append && (it.c == (it.n_keys - 1 - p.k_lo) / p.chunk);
   return it;
 }
 
@@ -709,7 +711,11 @@ cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t st) {
   p.Hkv = a.Hkv;
   p.n_keys = a.n_keys;
   p.chunk = a.chunk;
-  p.nchunks = decode_num_chunks(a.n_keys, a.chunk);
+  p.k_lo = a.k_lo;
+  p.append = a.append;
+  if (a.k_lo < 0 || a.k_lo % kTileKeys != 0 || a.k_lo >= a.n_keys || (a.k_lo > 0 && a.shift.on))
+    return cudaErrorInvalidValue;
+  p.nchunks = decode_num_chunks(a.n_keys - a.k_lo, a.chunk);
   p.item_base = 0;
   p.num_items = 0;
   p.scale_log2 = a.scale_log2;

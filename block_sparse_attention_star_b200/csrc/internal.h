@@ -115,6 +115,10 @@ struct AttnLaunch {
   SeqShift shift;         // per-sequence context lengths L + delta[s] (on = 0: all L)
   const void* anchor_k;   // mode 0: NULL (anchor keys are block 1's cached keys) or bf16 [B][n-1][Hkv][a][d]
   float scale_log2;
+  // A shard: blocks [blk0, blk0 + nblk) of every sequence (nblk = 0: through the last block).
+  // Mode 0: q and out hold the range's nblk * b rows per sequence.  Mode 1: parts are the
+  // range's chunks; the query tail is the last block's unless no_tail.
+  int blk0, nblk, no_tail;
 };
 int attn_num_parts(const AttnLaunch& a);  // mode 1: n * chunks_per_block
 cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t st, const char** why);
@@ -126,7 +130,9 @@ struct DecodeLaunch {
   const void* k_new;      // [B][Hkv][d] bf16 (pre-RoPE): appended at slot n_keys - 1 by the kernel
   const void* v_new;      // [B][Hkv][d] bf16
   const int32_t* pos;     // [B] position of the decoded token
-  int n_keys;             // keys [0, n_keys) of every sequence (the longest, with a shift)
+  int n_keys;             // keys [k_lo, n_keys) of every sequence (the longest, with a shift)
+  int k_lo;               // first key: 0, or a shard's first key (a multiple of 128; no shift then)
+  int append;             // 1: slot n_keys - 1 is the new token's, appended by the kernel
   SeqShift shift;         // sequence s has n_keys + delta[s] keys
   int chunk;              // keys per CTA
   CacheView cache;

@@ -256,6 +256,60 @@ int star_encode_layers(const star_shape* shape, int32_t n_layers, const star_cac
                        void* x, void* q, void* k, void* v, void* o, star_layer_fn fn, void* user,
                        star_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * Shards: Star Attention across several GPUs, one contiguous block range per GPU.
+ * The pages run one host per block ("Star Attention 完全拆解(一)", Phase 1: every host
+ * receives the anchor block c_1 with its own block; "仓库里的真实实现": only the host
+ * holding the last block appends the query and generated tokens' KV; "通信量:每层每
+ * token 一个标量加一个向量": per query token and layer each host contributes one
+ * (output, log-sum-exp) pair, which "组装全局结果" merges exactly).  Here a GPU owns
+ * blocks [block_begin, block_end) of every sequence; its partials are exchanged (an
+ * all-gather or a gather to the GPU that needs the output; the library leaves the
+ * transport to the caller's NCCL) and merged with star_lse_merge.
+ * The shape is the whole problem's (L = n*b, T_max); sequences must have one length
+ * (shape->seq_len NULL).  The cache of a shard holds its own blocks at their cache
+ * slots [block_begin*b, block_end*b), plus block 1's first a (anchor) tokens at slots
+ * [0, a) when block_begin > 0, plus the tail on the shard with block_end == n; its page
+ * table must cover all logical pages those occupy (the rest is never read).
+ * ------------------------------------------------------------------------- */
+typedef struct star_shard {
+  int32_t block_begin; /* first block of the range (0-based) */
+  int32_t block_end;   /* one past the last; 0 <= block_begin < block_end <= n */
+} star_shard;
+
+/* Phase 1 of a shard's blocks.  q: bf16 [B][R][Hq][d], k, v: bf16 [B][R][Hkv][d] and pos:
+ * int32 [B][R] for the range's R = (block_end - block_begin)*b context tokens;
+ * out: bf16 [B][R][Hq][d] (may be q; staging as in star_phase1_encode).  k_anchor,
+ * v_anchor: bf16 [B][a][Hkv][d] and pos_anchor: int32 [B][a], the anchor's tokens (block
+ * 1's first a), required when block_begin > 0 (ignored otherwise).  Writes the range's
+ * RoPE(K), V and, when block_begin > 0, the anchor's into the cache; the shard holding
+ * the last block also zeroes the tail slots.  Rows equal those of star_phase1_encode.
+ * Errors: those of star_phase1_encode; INVALID_ARG for a bad range. */
+int star_phase1_encode_shard(const star_shape* shape, const star_cache* cache, const star_shard* shard, const void* q,
+                             const void* k, const void* v, const int32_t* pos, const void* k_anchor,
+                             const void* v_anchor, const int32_t* pos_anchor, void* out, star_stream_t stream);
+
+/* Phase-2 partials of a shard's blocks: as star_phase2_partial, restricted to blocks
+ * [block_begin, block_end).  o_part: f32 [R_b][B][T][Hq][d], lse_part: f32 [R_b][B][T][Hq]
+ * with R_b = block_end - block_begin.  k, v (the query's, appended at [L, L+T)) only on the
+ * shard holding the last block, whose last partial includes the causal tail; NULL elsewhere.
+ * ws: star_workspace_size(STAR_OP_PHASE2, T) bytes.
+ * Errors: those of star_phase2_partial; INVALID_ARG for a bad range or k, v off the tail. */
+int star_phase2_partial_shard(const star_shape* shape, const star_cache* cache, const star_shard* shard, const void* q,
+                              const void* k, const void* v, const int32_t* q_pos, int32_t T, float* o_part,
+                              float* lse_part, void* ws, size_t ws_bytes, star_stream_t stream);
+
+/* One decode token's partial over a shard's keys: the range's context keys and, on the
+ * shard holding the last block, the tail up to and including the new token (its RoPE(k),
+ * v appended at cache slot cur_len there; k, v ignored elsewhere).  q: bf16 [B][1][Hq][d];
+ * pos: int32 [B] (the token's position, every shard).  o_part: f32 [B][Hq][d] (normalised
+ * local output), lse_part: f32 [B][Hq]; merging every shard's pair with star_lse_merge
+ * gives star_decode_step's output.  ws: star_workspace_size(STAR_OP_DECODE) bytes.
+ * Errors: those of star_decode_step; INVALID_ARG for a bad range. */
+int star_decode_partial_shard(const star_shape* shape, const star_cache* cache, const star_shard* shard, const void* q,
+                              const void* k, const void* v, const int32_t* pos, int32_t cur_len, float* o_part,
+                              float* lse_part, void* ws, size_t ws_bytes, star_stream_t stream);
+
 /* Tracing: when both are non-NULL (cudaEvent_t handles created by the caller),
  * every later call on this thread records `start_event` on its stream right
  * before launching its main kernel and `stop_event` right after it (Phase 1 and
