@@ -75,6 +75,10 @@ struct Params {
   int num_items;
   // Phase-1 anchor: its size, and whether its keys come from the tmKA map (roped at caller ids)
   int anchor, anchor_k_on;
+  // Block range [blk0, blk0 + nblk) of every sequence (a shard; the whole context by
+  // default); tail_on: the range holds the query tail.  Mode 0 reads q and writes out as
+  // rows [0, Lrows) per sequence, row r holding context token r + row_off.
+  int blk0, nblk, tail_on, row_off, Lrows;
   SeqShift sh;  // per-sequence context lengths L + delta[bi] (sh.on = 0: every sequence has L)
   float scale_log2;
 };
@@ -102,18 +106,20 @@ __device__ __forceinline__ Item decode_item(const Params& p, int idx) {
   if (MODE == 0) {
     const int nqt = p.b / kRows;
     const int npairs = p.G / 2;
-    const int per_group = p.n * nqt * npairs;
+    const int per_group = p.nblk * nqt * npairs;
     const int grp = idx / per_group;
     int w = idx - grp * per_group;
     it.bi = grp / p.Hkv;
     it.g = grp - it.bi * p.Hkv;
-    const int nonanchor = (p.n - 1) * nqt * npairs;
+    const int has_first = p.blk0 == 0;         // the range holds the context's first block
+    const int n_later = p.nblk - has_first;    // blocks with the anchor in front
+    const int nonanchor = n_later * nqt * npairs;
     int t, i;
     if (w < nonanchor) {
-      const int per_t = (p.n - 1) * npairs;
+      const int per_t = n_later * npairs;
       t = nqt - 1 - w / per_t;
       const int rem = w - (w / per_t) * per_t;
-      i = 1 + rem / npairs;
+      i = p.blk0 + has_first + rem / npairs;
       it.hp = rem - (rem / npairs) * npairs;
     } else {
       w -= nonanchor;
@@ -135,15 +141,15 @@ __device__ __forceinline__ Item decode_item(const Params& p, int idx) {
     it.g = rest % p.Hkv;
     rest /= p.Hkv;
     it.bi = rest % p.B;
-    const int c = rest / p.B;
+    const int c = p.blk0 * p.chunks_per_block + rest / p.B;  // the chunk's index in the context
     const int Ls = ctx_len(p, it.bi);
-    it.part = c;
+    it.part = c - p.blk0 * p.chunks_per_block;
     // The chunk's context keys, cut at the sequence's length; the tail (query tokens,
     // cache indices Ls ..) follows the chunk that holds the last context key.
     it.a_start = c * p.chunk_keys;
     it.a_end = min(it.a_start + p.chunk_keys, Ls);
     it.a_tiles = it.a_end > it.a_start ? (it.a_end - it.a_start + kKeys - 1) / kKeys : 0;
-    const bool last = (c == (Ls - 1) / p.chunk_keys);
+    const bool last = p.tail_on && (c == (Ls - 1) / p.chunk_keys);
     it.b_start = Ls;
     it.b_tiles = last ? (Ls % kKeys + p.Ntok + kKeys - 1) / kKeys : 0;
     it.r0 = 0;
@@ -352,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int h = 0; h < D / 64; ++h)
             tma_load_4d(smem + S::kQ0 + w * S::kTile + h * (kRows * 128), &tmQ, &q_full[w], h * 64,
-                        it.g * p.G + 2 * it.hp + w, it.r0, it.bi);
+                        it.g * p.G + 2 * it.hp + w, it.r0 - p.row_off, it.bi);
         }
         ++qc;
       }
@@ -616,7 +622,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const RowInfo ri = row_info<MODE>(p, it, wg, row);
       const float inv_l = (lr > 0.f) ? 1.f / lr : 0.f;
       if (MODE == 0) {
-        bf16* dst = p.out_bf16 + (((size_t)it.bi * p.L + ri.tok) * p.Hq + ri.head) * D;
+        bf16* dst = p.out_bf16 + (((size_t)it.bi * p.Lrows + (ri.tok - p.row_off)) * p.Hq + ri.head) * D;
         const bool keep = ri.tok < ctx_len(p, it.bi);  // rows past a shorter sequence are padding
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
@@ -778,8 +784,17 @@ cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t st, const char** 
   p.n = a.n;
   p.Ntok = a.Ntok;
   p.scale_log2 = a.scale_log2;
+  p.blk0 = a.blk0;
+  p.nblk = a.nblk ? a.nblk : a.n - a.blk0;
+  p.tail_on = a.blk0 + p.nblk == a.n && !a.no_tail;
+  p.row_off = a.mode == 0 ? a.blk0 * a.b : 0;
+  p.Lrows = a.mode == 0 ? p.nblk * a.b : 0;
+  if (a.blk0 < 0 || p.nblk < 1 || a.blk0 + p.nblk > a.n) {
+    if (why) *why = "block range outside the context";
+    return cudaErrorInvalidValue;
+  }
   if (a.mode == 0) {
-    p.num_items = a.B * a.Hkv * a.n * (a.b / kRows) * (p.G / 2);
+    p.num_items = a.B * a.Hkv * p.nblk * (a.b / kRows) * (p.G / 2);
   } else {
     p.chunks_per_block = a.chunks_per_block;
     p.chunk_keys = a.b / a.chunks_per_block;
@@ -789,7 +804,7 @@ cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t st, const char** 
     p.NTT = (a.Ntok + p.TQ - 1) / p.TQ;
     p.NHT = (p.G + p.HT - 1) / p.HT;
     p.npairs = (p.NTT * p.NHT + 1) / 2;
-    p.num_items = a.n * a.chunks_per_block * a.B * a.Hkv * p.npairs;
+    p.num_items = p.nblk * a.chunks_per_block * a.B * a.Hkv * p.npairs;
   }
   CUtensorMap mk, mv;
   if (!make_pool_map(&mk, a.cache.k_pool, a.d, a.cache.P, a.Hkv, a.cache.num_pages) ||
@@ -798,7 +813,7 @@ cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t st, const char** 
     return cudaErrorInvalidValue;
   }
   CUtensorMap mq = mk;  // mode 1 stages Q with its own threads; the map is unused there
-  if (a.mode == 0 && !make_q_map(&mq, a.q, a.d, a.Hq, a.L, a.B)) {
+  if (a.mode == 0 && !make_q_map(&mq, a.q, a.d, a.Hq, p.Lrows, a.B)) {
     if (why) *why = "cuTensorMapEncodeTiled failed for the rotated queries";
     return cudaErrorInvalidValue;
   }
