@@ -107,11 +107,13 @@ def test_build_positions_bit_exact():
             assert np.array_equal(bmap[bi].cpu().numpy(), want_map)
 
 
-def test_lse_merge_edge_cases():
+@pytest.mark.parametrize("n", [5, 37, 64])
+def test_lse_merge_edge_cases(n):
+    """n = 5: one warp per row; 37 and 64 partials: the decode-sized variant (two warps per row)."""
     import block_sparse_attention_star_b200 as star
-    rng = np.random.default_rng(5)
+    rng = np.random.default_rng(5 + n)
     for d in (64, 128):
-        n, rows = 5, 300
+        rows = 300
         O = rng.standard_normal((n, rows, d)).astype(np.float32)
         L = (rng.standard_normal((n, rows)) * 20).astype(np.float32)
         L[1, :50] = -np.inf                  # empty blocks
