@@ -275,6 +275,19 @@ class ShardRun:
         self.o_dec = torch.empty((wl.S, wl.B, wl.Hq, wl.d), dtype=torch.bfloat16, device=device)
         self.lse_dec = torch.empty((wl.S, wl.B, wl.Hq), dtype=torch.float32, device=device)
 
+    def launches_per_step(self) -> int:
+        """Library kernel launches of one step on this rank.  Phase 1: RoPE + KV append of the
+        range, of the anchor (a range after block 1), the tail zero-fill (the last range),
+        RoPE(Q), attention.  Phase 2: the query's KV append (last range), RoPE(Q), attention,
+        the chunk merge (when blocks are split into chunks), the exchange's merge.  Per decode
+        step: the decode kernel, its chunk merge, the exchange's merge."""
+        wl, star = self.wl, self.star
+        q_bytes = -(-wl.B * wl.T * wl.Hq * wl.d * 2 // 256) * 256
+        chunked = star.star_workspace_size(self.shape, star.STAR_OP_PHASE2, wl.T) > q_bytes
+        p1 = 3 + (1 if self.ex.begin > 0 else 0) + (1 if self.tail else 0)
+        p2 = 2 + (1 if self.tail else 0) + (1 if chunked else 0) + 1
+        return p1 + p2 + 3 * wl.S
+
     def step(self):
         s, wl, c, sh = self.star, self.wl, self.ctx, self.ex.shard()
         s.star_phase1_encode_shard(self.shape, self.cache, sh, c["q_ctx"], c["k_ctx"], c["v_ctx"], c["pos_ctx"],
@@ -331,6 +344,7 @@ def run_shard(args, rank, world, local_rank):
             "config": dict(workload_config(wl, world), parallelism=f"context blocks sharded over {world} GPUs"),
             "exchange": f"per query call and per decode step: all-gather of the f32 (O, LSE) partials "
                         f"(rank 0 holds {nl} of {wl.n} blocks), then star_lse_merge on every rank",
+            "gpu_launches": run.launches_per_step() * K,
             "device_status": status, "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)
