@@ -57,7 +57,9 @@ int check_shape(const star_shape* s) {
     return fail(STAR_ERR_UNSUPPORTED_SHAPE, "GQA group size Hq/Hkv = %d is not supported (2, 4 or 8)", G);
   if (s->d != 64 && s->d != 128) return fail(STAR_ERR_UNSUPPORTED_SHAPE, "head dim %d is not supported (64 or 128)", s->d);
   if ((int64_t)s->n * s->b != s->L)
-    return fail(STAR_ERR_UNSUPPORTED_SHAPE, "L (%d) must equal n*b (%d*%d): ragged last blocks are not supported",
+    return fail(STAR_ERR_UNSUPPORTED_SHAPE,
+                "L (%d) must equal n*b (%d*%d): L is the capacity; shorter contexts (a ragged last block) "
+                "go through seq_len",
                 s->L, s->n, s->b);
   if (s->b % 128) return fail(STAR_ERR_UNSUPPORTED_SHAPE, "block size b (%d) must be a multiple of 128", s->b);
   if (s->page_tokens % 128) return fail(STAR_ERR_UNSUPPORTED_SHAPE, "page_tokens (%d) must be a multiple of 128", s->page_tokens);
