@@ -58,6 +58,9 @@ def parse_args():
     ap.add_argument("--shard", action="store_true",
                     help="multi-GPU Star Attention: every rank owns a block range of the same sequences "
                          "(Phase 1 on its blocks, Phase-2 and decode partials exchanged and merged)")
+    ap.add_argument("--exchange", default="p2p", choices=["p2p", "nccl"],
+                    help="--shard: partials all-gathered by NCCL, or pushed by the kernels into every GPU's "
+                         "exchange buffer over peer memory")
     ap.add_argument("--layers", type=int, default=0,
                     help="time N layers of context encoding (star_encode_layers, random projections) instead")
     return ap.parse_args()
@@ -245,9 +248,9 @@ class ShardRun:
     its block range of every sequence (the same sequences on every rank), the anchor's
     tokens when the range does not hold block 1, and the tail on the rank with the last block."""
 
-    def __init__(self, wl, device):
+    def __init__(self, wl, device, exchange="p2p"):
         import block_sparse_attention_star_b200 as star
-        from block_sparse_attention_star_b200.shard import ShardExchange
+        from block_sparse_attention_star_b200.shard import PeerExchange, ShardExchange
         self.star, self.wl, self.dev = star, wl, device
         inp = make_inputs(wl, device)
         self.shape = workload_shape(wl)
@@ -274,6 +277,11 @@ class ShardRun:
         self.pl = torch.empty((1, wl.B, wl.Hq), dtype=torch.float32, device=device)
         self.o_dec = torch.empty((wl.S, wl.B, wl.Hq, wl.d), dtype=torch.bfloat16, device=device)
         self.lse_dec = torch.empty((wl.S, wl.B, wl.Hq), dtype=torch.float32, device=device)
+        self.p2p = exchange == "p2p"
+        if self.p2p:
+            self.pq = PeerExchange(wl.B * wl.T * wl.Hq, wl.d, self.ex.nmax, device=device)
+            self.pd = PeerExchange(wl.B * wl.Hq, wl.d, 1, device=device)
+            self.ws2p = star.workspace(self.shape, star.STAR_OP_PHASE2_PUSH, wl.T, device)
 
     def launches_per_step(self) -> int:
         """Library kernel launches of one step on this rank.  Phase 1: RoPE + KV append of the
@@ -285,6 +293,8 @@ class ShardRun:
         q_bytes = -(-wl.B * wl.T * wl.Hq * wl.d * 2 // 256) * 256
         chunked = star.star_workspace_size(self.shape, star.STAR_OP_PHASE2, wl.T) > q_bytes
         p1 = 3 + (1 if self.ex.begin > 0 else 0) + (1 if self.tail else 0)
+        if self.p2p:  # attention + push (merge-scatter) + the exchange merge; decode: kernel, push, merge
+            return p1 + 2 + (1 if self.tail else 0) + 2 + 3 * wl.S
         p2 = 2 + (1 if self.tail else 0) + (1 if chunked else 0) + 1
         return p1 + p2 + 3 * wl.S
 
@@ -293,12 +303,24 @@ class ShardRun:
         s.star_phase1_encode_shard(self.shape, self.cache, sh, c["q_ctx"], c["k_ctx"], c["v_ctx"], c["pos_ctx"],
                                    self.anchor["k_ctx"], self.anchor["v_ctx"], self.anchor["pos_ctx"], self.o_ctx)
         q = self.query
+        d = self.dec
+        if self.p2p:
+            # The kernels push every partial into each GPU's exchange buffer; each GPU merges its own.
+            s.star_phase2_partial_shard_push(self.shape, self.cache, sh, q["q_query"],
+                                             q["k_query"] if self.tail else None, q["v_query"] if self.tail else None,
+                                             q["pos_query"], wl.T, self.pq.ex, self.pq.next_epoch(), self.ws2p)
+            self.pq.merge(self.o_q, self.lse_q)
+            for st in range(wl.S):
+                s.star_decode_partial_shard_push(self.shape, self.cache, sh, d["q_dec"][st], d["k_dec"][st],
+                                                 d["v_dec"][st], d["pos_dec"][st], wl.L + wl.T + st, self.pd.ex,
+                                                 self.pd.next_epoch(), self.wsd)
+                self.pd.merge(self.o_dec[st], self.lse_dec[st])
+            return
         s.star_phase2_partial_shard(self.shape, self.cache, sh, q["q_query"], q["k_query"] if self.tail else None,
                                     q["v_query"] if self.tail else None, q["pos_query"], wl.T, self.o_part,
                                     self.lse_part, self.ws2)
         rows = wl.B * wl.T * wl.Hq
         self.ex.gather_merge(self.o_part.view(-1, rows, wl.d), self.lse_part.view(-1, rows), self.o_q, self.lse_q)
-        d = self.dec
         for st in range(wl.S):
             s.star_decode_partial_shard(self.shape, self.cache, sh, d["q_dec"][st], d["k_dec"][st], d["v_dec"][st],
                                         d["pos_dec"][st], wl.L + wl.T + st, self.po[0], self.pl[0], self.wsd)
@@ -313,7 +335,7 @@ def run_shard(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     wl = get_config(args.config)
-    run = ShardRun(wl, dev)
+    run = ShardRun(wl, dev, args.exchange)
     for _ in range(max(3, args.warmup)):
         run.step()
     torch.cuda.synchronize()
@@ -342,8 +364,11 @@ def run_shard(args, rank, world, local_rank):
             "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) bf16; 1% of context key rows x8 where the workload says peaky)",
             "config": dict(workload_config(wl, world), parallelism=f"context blocks sharded over {world} GPUs"),
-            "exchange": f"per query call and per decode step: all-gather of the f32 (O, LSE) partials "
-                        f"(rank 0 holds {nl} of {wl.n} blocks), then star_lse_merge on every rank",
+            "exchange": (f"per query call and per decode step: the partial kernels push the f32 (O, LSE) "
+                         f"partials into every GPU's exchange buffer over peer memory; each GPU merges its own "
+                         f"(rank 0 holds {nl} of {wl.n} blocks)") if run.p2p else
+                        (f"per query call and per decode step: all-gather of the f32 (O, LSE) partials "
+                         f"(rank 0 holds {nl} of {wl.n} blocks), then star_lse_merge on every rank"),
             "gpu_launches": run.launches_per_step() * K,
             "device_status": status, "clocks": clk.summary(),
         }

@@ -38,7 +38,7 @@ STAR_ERR_CUDA = -5
 STAR_ERR_TIMEOUT = -6
 STAR_ERR_CALLBACK = -7
 STAR_LAYER_QKV, STAR_LAYER_OUT = 0, 1
-STAR_OP_PHASE1, STAR_OP_PHASE2, STAR_OP_DECODE, STAR_OP_PHASE1_ANCHOR = 1, 2, 3, 4
+STAR_OP_PHASE1, STAR_OP_PHASE2, STAR_OP_DECODE, STAR_OP_PHASE1_ANCHOR, STAR_OP_PHASE2_PUSH = 1, 2, 3, 4, 5
 STAR_DEBUG_SKIP_FIRST_LOAD = 1
 
 
@@ -75,6 +75,12 @@ class StarShape(ctypes.Structure):
 class StarShard(ctypes.Structure):
     """Blocks [block_begin, block_end) of every sequence, owned by one GPU (star.h star_shard)."""
     _fields_ = [("block_begin", ctypes.c_int32), ("block_end", ctypes.c_int32)]
+
+
+class StarExchange(ctypes.Structure):
+    """One rank's view of the peer-memory exchange (star.h star_exchange)."""
+    _fields_ = [("world", ctypes.c_int32), ("rank", ctypes.c_int32), ("slots", ctypes.c_int32),
+                ("peers", ctypes.c_void_p * 8)]
 
 
 class StarCache(ctypes.Structure):
@@ -123,6 +129,15 @@ def lib() -> ctypes.CDLL:
                                           ctypes.c_int),
             "star_decode_partial_shard": ([P(StarShape), P(StarCache), P(StarShard), V, V, V, V, I32, V, V, V, SZ, V],
                                           ctypes.c_int),
+            "star_exchange_size": ([I32, I32, I64, I32, P(SZ)], ctypes.c_int),
+            "star_phase2_partial_shard_push": ([P(StarShape), P(StarCache), P(StarShard), V, V, V, V, I32,
+                                                P(StarExchange), ctypes.c_uint64, V, SZ, V], ctypes.c_int),
+            "star_decode_partial_shard_push": ([P(StarShape), P(StarCache), P(StarShard), V, V, V, V, I32,
+                                                P(StarExchange), ctypes.c_uint64, V, SZ, V], ctypes.c_int),
+            "star_exchange_merge": ([P(StarExchange), I64, I32, ctypes.c_uint64, V, V, V], ctypes.c_int),
+            "star_ipc_export": ([V, V, P(ctypes.c_uint64)], ctypes.c_int),
+            "star_ipc_open": ([V, ctypes.c_uint64, P(V)], ctypes.c_int),
+            "star_ipc_close": ([V, ctypes.c_uint64], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -353,6 +368,55 @@ def star_decode_partial_shard(shape, cache: PagedKVCache, shard: StarShard, q, k
                                            _ptr(o_part, "o_part", torch.float32),
                                            _ptr(lse_part, "lse_part", torch.float32), _ptr(ws, "ws"),
                                            ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def star_exchange_size(world: int, slots: int, rows: int, d: int) -> int:
+    out = ctypes.c_size_t()
+    _check(lib().star_exchange_size(world, slots, rows, d, ctypes.byref(out)))
+    return out.value
+
+
+def star_phase2_partial_shard_push(shape, cache: PagedKVCache, shard: StarShard, q, k, v, q_pos, T: int,
+                                   ex: StarExchange, epoch: int, ws, stream=None):
+    _check(lib().star_phase2_partial_shard_push(ctypes.byref(shape), ctypes.byref(cache.c), ctypes.byref(shard),
+                                                _ptr(q, "q", torch.bfloat16), _ptr(k, "k", torch.bfloat16),
+                                                _ptr(v, "v", torch.bfloat16), _ptr(q_pos, "q_pos", torch.int32), T,
+                                                ctypes.byref(ex), epoch, _ptr(ws, "ws"),
+                                                ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def star_decode_partial_shard_push(shape, cache: PagedKVCache, shard: StarShard, q, k, v, pos, cur_len: int,
+                                   ex: StarExchange, epoch: int, ws, stream=None):
+    _check(lib().star_decode_partial_shard_push(ctypes.byref(shape), ctypes.byref(cache.c), ctypes.byref(shard),
+                                                _ptr(q, "q", torch.bfloat16), _ptr(k, "k", torch.bfloat16),
+                                                _ptr(v, "v", torch.bfloat16), _ptr(pos, "pos", torch.int32), cur_len,
+                                                ctypes.byref(ex), epoch, _ptr(ws, "ws"),
+                                                ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def star_exchange_merge(ex: StarExchange, rows: int, d: int, epoch: int, out, lse_out=None, stream=None):
+    _check(lib().star_exchange_merge(ctypes.byref(ex), rows, d, epoch, _ptr(out, "out", torch.bfloat16),
+                                     _ptr(lse_out, "lse_out", torch.float32), _stream(stream)))
+
+
+def star_ipc_export(t: torch.Tensor) -> tuple[bytes, int]:
+    """(64-byte IPC handle, offset) of a device tensor's memory, for another process to open."""
+    h = (ctypes.c_ubyte * 64)()
+    off = ctypes.c_uint64()
+    _check(lib().star_ipc_export(ctypes.c_void_p(t.data_ptr()), h, ctypes.byref(off)))
+    return bytes(h), off.value
+
+
+def star_ipc_open(handle: bytes, offset: int) -> int:
+    """Device address, valid in this process, of memory another process exported."""
+    h = (ctypes.c_ubyte * 64).from_buffer_copy(handle)
+    ptr = ctypes.c_void_p()
+    _check(lib().star_ipc_open(h, offset, ctypes.byref(ptr)))
+    return ptr.value
+
+
+def star_ipc_close(ptr: int, offset: int) -> None:
+    _check(lib().star_ipc_close(ctypes.c_void_p(ptr), offset))
 
 
 def star_debug_set(wait_limit_ns: int = 0, flags: int = 0) -> None:

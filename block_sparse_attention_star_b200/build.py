@@ -14,7 +14,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libstar.so")
-SOURCES = ["api.cu", "attn_sm100.cu", "rope_append.cu", "merge.cu", "decode.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "attn_sm100.cu", "rope_append.cu", "merge.cu", "decode.cu", "noalloc.cu", "exchange.cu"]
 HEADERS = ["common.cuh", "internal.h"]
 
 

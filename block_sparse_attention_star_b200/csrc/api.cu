@@ -183,6 +183,16 @@ size_t phase2_ws_bytes(const star_shape* s, int T) {
   return qb + round_up(parts * rows * s->d * sizeof(float), 256) + round_up(parts * rows * sizeof(float), 256);
 }
 
+// The push variant of the Phase-2 shard always stages the chunk partials (merged into the
+// exchange slots by the scatter kernel), even with one chunk per block.
+size_t phase2_push_ws_bytes(const star_shape* s, int T) {
+  const int cpb = phase2_chunks_per_block(s, T);
+  const size_t rows = (size_t)s->B * T * s->Hq;
+  const size_t parts = (size_t)s->n * cpb;
+  return phase2_q_bytes(s, T) + round_up(parts * rows * s->d * sizeof(float), 256) +
+         round_up(parts * rows * sizeof(float), 256);
+}
+
 int anchor_of(const star_shape* s) { return s->anchor ? s->anchor : s->b; }
 
 // Per-sequence context lengths as shifts of the capacity frame (delta = L_s - L).
@@ -269,6 +279,10 @@ int star_workspace_size(const star_shape* shape, int op, int32_t T, size_t* byte
       return STAR_OK;
     case STAR_OP_DECODE: *bytes_out = decode_ws_bytes(shape); return STAR_OK;
     case STAR_OP_PHASE1_ANCHOR: *bytes_out = anchor_ws_bytes(shape); return STAR_OK;
+    case STAR_OP_PHASE2_PUSH:
+      if (T <= 0 || T > shape->T_max) return fail(STAR_ERR_INVALID_ARG, "T (%d) must be in [1, T_max=%d]", T, shape->T_max);
+      *bytes_out = phase2_push_ws_bytes(shape, T);
+      return STAR_OK;
     default: return fail(STAR_ERR_INVALID_ARG, "unknown op %d", op);
   }
 }
@@ -616,22 +630,54 @@ int star_phase1_encode_shard(const star_shape* shape, const star_cache* cache, c
   return STAR_OK;
 }
 
-int star_phase2_partial_shard(const star_shape* shape, const star_cache* cache, const star_shard* shard, const void* q,
-                              const void* k, const void* v, const int32_t* q_pos, int32_t T, float* o_part,
-                              float* lse_part, void* ws, size_t ws_bytes, star_stream_t stream) {
+static int check_exchange(const star_exchange* ex, int min_slots) {
+  if (!ex) return fail(STAR_ERR_INVALID_ARG, "exchange is NULL");
+  if (ex->world < 1 || ex->world > 8) return fail(STAR_ERR_UNSUPPORTED_SHAPE, "exchange world %d outside [1, 8]", ex->world);
+  if (ex->rank < 0 || ex->rank >= ex->world)
+    return fail(STAR_ERR_INVALID_ARG, "exchange rank %d outside [0, %d)", ex->rank, ex->world);
+  if (ex->slots < min_slots || ex->slots < 1)
+    return fail(STAR_ERR_CAPACITY, "exchange holds %d partials per rank, %d needed", ex->slots, min_slots);
+  for (int w = 0; w < ex->world; ++w) {
+    if (!ex->peers[w]) return fail(STAR_ERR_INVALID_ARG, "exchange peers[%d] is NULL", w);
+    if (reinterpret_cast<uintptr_t>(ex->peers[w]) & 255u)
+      return fail(STAR_ERR_ALIGNMENT, "exchange peers[%d] is not 256-byte aligned", w);
+  }
+  return STAR_OK;
+}
+
+static star::ExchangeView exchange_view(const star_exchange* ex) {
+  star::ExchangeView x;
+  memset(&x, 0, sizeof(x));
+  x.world = ex->world;
+  x.rank = ex->rank;
+  x.slots = ex->slots;
+  for (int w = 0; w < ex->world; ++w) x.peers[w] = ex->peers[w];
+  return x;
+}
+
+// Phase-2 partials of a shard; ex == NULL: into o_part / lse_part, else pushed into the
+// exchange slots of every rank (epoch).
+static int phase2_shard(const star_shape* shape, const star_cache* cache, const star_shard* shard, const void* q,
+                        const void* k, const void* v, const int32_t* q_pos, int32_t T, float* o_part, float* lse_part,
+                        const star_exchange* ex, uint64_t epoch, void* ws, size_t ws_bytes, star_stream_t stream) {
   int rc = check_shape(shape);
   if (!rc) rc = check_cache(shape, cache);
   if (!rc) rc = check_shard(shape, shard);
+  if (!rc && ex) rc = check_exchange(ex, shard->block_end - shard->block_begin);
   if (rc) return rc;
   STAR_REQUIRE_PTR(q, "q");
   STAR_REQUIRE_PTR4(q_pos, "q_pos");
-  STAR_REQUIRE_PTR(o_part, "o_part");
-  STAR_REQUIRE_PTR4(lse_part, "lse_part");
+  if (!ex) {
+    STAR_REQUIRE_PTR(o_part, "o_part");
+    STAR_REQUIRE_PTR4(lse_part, "lse_part");
+  } else if (epoch == 0) {
+    return fail(STAR_ERR_INVALID_ARG, "exchange epochs start at 1");
+  }
   if ((k == nullptr) != (v == nullptr)) return fail(STAR_ERR_INVALID_ARG, "k and v must both be given or both be NULL");
   if (T <= 0 || T > shape->T_max) return fail(STAR_ERR_INVALID_ARG, "T (%d) must be in [1, T_max=%d]", T, shape->T_max);
   const bool tail = shard->block_end == shape->n;
   if (k && !tail) return fail(STAR_ERR_INVALID_ARG, "only the shard holding the last block appends the query's k, v");
-  const size_t need = phase2_ws_bytes(shape, T);
+  const size_t need = ex ? phase2_push_ws_bytes(shape, T) : phase2_ws_bytes(shape, T);
   STAR_REQUIRE_PTR(ws, "ws");
   if (ws_bytes < need) return fail(STAR_ERR_CAPACITY, "workspace %zu bytes < %zu needed", ws_bytes, need);
   cudaStream_t st = (cudaStream_t)stream;
@@ -651,7 +697,7 @@ int star_phase2_partial_shard(const star_shape* shape, const star_cache* cache, 
   char* chunk_ws = reinterpret_cast<char*>(ws) + phase2_q_bytes(shape, T);
   float* o_dst = o_part;
   float* l_dst = lse_part;
-  if (cpb > 1) {
+  if (cpb > 1 || ex) {
     o_dst = reinterpret_cast<float*>(chunk_ws);
     l_dst = reinterpret_cast<float*>(chunk_ws + round_up(parts * rows * shape->d * sizeof(float), 256));
   }
@@ -681,23 +727,47 @@ int star_phase2_partial_shard(const star_shape* shape, const star_cache* cache, 
   if (e == cudaSuccess) e = star::launch_attention(a, st, &why);
   trace_end(st);
   if (e != cudaSuccess) return why ? fail(STAR_ERR_CUDA, "%s", why) : cuda_fail(e, "phase2 shard attention launch");
-  if (cpb > 1) {
+  if (ex) {
+    e = star::launch_merge_scatter(exchange_view(ex), nblk, cpb, (long long)rows, shape->d, o_dst, l_dst,
+                                   (unsigned long long)epoch, st);
+    if (e != cudaSuccess) return cuda_fail(e, "phase2 shard push");
+  } else if (cpb > 1) {
     e = star::launch_lse_merge(nblk, cpb, (int64_t)rows, shape->d, o_dst, l_dst, o_part, false, lse_part, st);
     if (e != cudaSuccess) return cuda_fail(e, "phase2 shard chunk merge");
   }
   return STAR_OK;
 }
 
-int star_decode_partial_shard(const star_shape* shape, const star_cache* cache, const star_shard* shard, const void* q,
-                              const void* k, const void* v, const int32_t* pos, int32_t cur_len, float* o_part,
+int star_phase2_partial_shard(const star_shape* shape, const star_cache* cache, const star_shard* shard, const void* q,
+                              const void* k, const void* v, const int32_t* q_pos, int32_t T, float* o_part,
                               float* lse_part, void* ws, size_t ws_bytes, star_stream_t stream) {
+  return phase2_shard(shape, cache, shard, q, k, v, q_pos, T, o_part, lse_part, nullptr, 0, ws, ws_bytes, stream);
+}
+
+int star_phase2_partial_shard_push(const star_shape* shape, const star_cache* cache, const star_shard* shard,
+                                   const void* q, const void* k, const void* v, const int32_t* q_pos, int32_t T,
+                                   const star_exchange* ex, uint64_t epoch, void* ws, size_t ws_bytes,
+                                   star_stream_t stream) {
+  if (!ex) return fail(STAR_ERR_INVALID_ARG, "exchange is NULL");
+  return phase2_shard(shape, cache, shard, q, k, v, q_pos, T, nullptr, nullptr, ex, epoch, ws, ws_bytes, stream);
+}
+
+static int decode_shard(const star_shape* shape, const star_cache* cache, const star_shard* shard, const void* q,
+                        const void* k, const void* v, const int32_t* pos, int32_t cur_len, float* o_part,
+                        float* lse_part, const star_exchange* ex, uint64_t epoch, void* ws, size_t ws_bytes,
+                        star_stream_t stream) {
   int rc = check_shape(shape);
   if (!rc) rc = check_cache(shape, cache);
   if (!rc) rc = check_shard(shape, shard);
+  if (!rc && ex) rc = check_exchange(ex, 1);
   if (rc) return rc;
   STAR_REQUIRE_PTR(q, "q");
-  STAR_REQUIRE_PTR4(o_part, "o_part");
-  STAR_REQUIRE_PTR4(lse_part, "lse_part");
+  if (!ex) {
+    STAR_REQUIRE_PTR4(o_part, "o_part");
+    STAR_REQUIRE_PTR4(lse_part, "lse_part");
+  } else if (epoch == 0) {
+    return fail(STAR_ERR_INVALID_ARG, "exchange epochs start at 1");
+  }
   STAR_REQUIRE_PTR(ws, "ws");
   const bool tail = shard->block_end == shape->n;
   if (tail) {
@@ -746,8 +816,93 @@ int star_decode_partial_shard(const star_shape* shape, const star_cache* cache, 
   cudaError_t e = star::launch_decode(a, st);
   trace_end(st);
   if (e != cudaSuccess) return cuda_fail(e, "decode shard launch");
+  if (ex) {
+    e = star::launch_merge_scatter(exchange_view(ex), 1, nch, (long long)rows, shape->d, a.o_ws, a.lse_ws,
+                                   (unsigned long long)epoch, st);
+    return e == cudaSuccess ? STAR_OK : cuda_fail(e, "decode shard push");
+  }
   e = star::launch_lse_merge(1, nch, (int64_t)rows, shape->d, a.o_ws, a.lse_ws, o_part, false, lse_part, st);
   return e == cudaSuccess ? STAR_OK : cuda_fail(e, "decode shard merge launch");
+}
+
+int star_decode_partial_shard(const star_shape* shape, const star_cache* cache, const star_shard* shard, const void* q,
+                              const void* k, const void* v, const int32_t* pos, int32_t cur_len, float* o_part,
+                              float* lse_part, void* ws, size_t ws_bytes, star_stream_t stream) {
+  return decode_shard(shape, cache, shard, q, k, v, pos, cur_len, o_part, lse_part, nullptr, 0, ws, ws_bytes, stream);
+}
+
+int star_decode_partial_shard_push(const star_shape* shape, const star_cache* cache, const star_shard* shard,
+                                   const void* q, const void* k, const void* v, const int32_t* pos, int32_t cur_len,
+                                   const star_exchange* ex, uint64_t epoch, void* ws, size_t ws_bytes,
+                                   star_stream_t stream) {
+  if (!ex) return fail(STAR_ERR_INVALID_ARG, "exchange is NULL");
+  return decode_shard(shape, cache, shard, q, k, v, pos, cur_len, nullptr, nullptr, ex, epoch, ws, ws_bytes, stream);
+}
+
+int star_exchange_size(int32_t world, int32_t slots, int64_t rows, int32_t d, size_t* bytes_out) {
+  if (!bytes_out) return fail(STAR_ERR_INVALID_ARG, "bytes_out is NULL");
+  if (world < 1 || world > 8) return fail(STAR_ERR_UNSUPPORTED_SHAPE, "exchange world %d outside [1, 8]", world);
+  if (slots < 1 || rows < 1) return fail(STAR_ERR_INVALID_ARG, "slots and rows must be positive");
+  if (d != 64 && d != 128) return fail(STAR_ERR_UNSUPPORTED_SHAPE, "head dim %d is not supported (64 or 128)", d);
+  *bytes_out = star::exchange_bytes(world, slots, (long long)rows, d);
+  return STAR_OK;
+}
+
+int star_exchange_merge(const star_exchange* ex, int64_t rows, int32_t d, uint64_t epoch, void* out, float* lse_out,
+                        star_stream_t stream) {
+  int rc = check_exchange(ex, 1);
+  if (rc) return rc;
+  if (rows < 1) return fail(STAR_ERR_INVALID_ARG, "rows must be positive");
+  if (d != 64 && d != 128) return fail(STAR_ERR_UNSUPPORTED_SHAPE, "head dim %d is not supported (64 or 128)", d);
+  if (epoch == 0) return fail(STAR_ERR_INVALID_ARG, "exchange epochs start at 1");
+  STAR_REQUIRE_PTR(out, "out");
+  if (lse_out && (reinterpret_cast<uintptr_t>(lse_out) & 3u)) return fail(STAR_ERR_ALIGNMENT, "lse_out is not 4-byte aligned");
+  cudaError_t e = star::launch_gather_merge(exchange_view(ex), (long long)rows, d, (unsigned long long)epoch, out,
+                                            lse_out, (cudaStream_t)stream);
+  return e == cudaSuccess ? STAR_OK : cuda_fail(e, "exchange merge launch");
+}
+
+typedef CUresult (*GetAddressRangeFn)(CUdeviceptr*, size_t*, CUdeviceptr);
+
+int star_ipc_export(const void* ptr, void* handle_out, uint64_t* offset_out) {
+  if (!ptr || !handle_out || !offset_out) return fail(STAR_ERR_INVALID_ARG, "NULL argument");
+  static GetAddressRangeFn range = nullptr;
+  if (!range) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return fail(STAR_ERR_CUDA, "cuMemGetAddressRange is not available");
+    range = reinterpret_cast<GetAddressRangeFn>(fn);
+  }
+  CUdeviceptr base = 0;
+  size_t size = 0;
+  if (range(&base, &size, reinterpret_cast<CUdeviceptr>(ptr)) != CUDA_SUCCESS)
+    return fail(STAR_ERR_INVALID_ARG, "pointer is not device memory of this process");
+  cudaIpcMemHandle_t h;
+  cudaError_t e = cudaIpcGetMemHandle(&h, reinterpret_cast<void*>(base));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaIpcGetMemHandle");
+  static_assert(sizeof(h) == 64, "IPC handle size");
+  memcpy(handle_out, &h, sizeof(h));
+  *offset_out = (uint64_t)(reinterpret_cast<CUdeviceptr>(ptr) - base);
+  return STAR_OK;
+}
+
+int star_ipc_open(const void* handle, uint64_t offset, void** ptr_out) {
+  if (!handle || !ptr_out) return fail(STAR_ERR_INVALID_ARG, "NULL argument");
+  cudaIpcMemHandle_t h;
+  memcpy(&h, handle, sizeof(h));
+  void* base = nullptr;
+  cudaError_t e = cudaIpcOpenMemHandle(&base, h, cudaIpcMemLazyEnablePeerAccess);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaIpcOpenMemHandle");
+  *ptr_out = reinterpret_cast<char*>(base) + offset;
+  return STAR_OK;
+}
+
+int star_ipc_close(void* ptr, uint64_t offset) {
+  if (!ptr) return fail(STAR_ERR_INVALID_ARG, "ptr is NULL");
+  cudaError_t e = cudaIpcCloseMemHandle(reinterpret_cast<char*>(ptr) - offset);
+  return e == cudaSuccess ? STAR_OK : cuda_fail(e, "cudaIpcCloseMemHandle");
 }
 
 int star_set_trace_events(void* start_event, void* stop_event) {
@@ -762,7 +917,8 @@ int star_device_status(star_stream_t stream, int32_t* status_out) {
   int code = 0;
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   cudaError_t (*readers[])(int*) = {star::read_and_clear_error_attn, star::read_and_clear_error_decode,
-                                   star::read_and_clear_error_rope, star::read_and_clear_error_merge};
+                                   star::read_and_clear_error_rope, star::read_and_clear_error_merge,
+                                   star::read_and_clear_error_exchange};
   for (auto rd : readers) {
     if (e != cudaSuccess) break;
     int c = 0;
@@ -784,6 +940,7 @@ int star_debug_set(uint64_t wait_limit_ns, int32_t flags) {
   const int dev_flags = (flags & STAR_DEBUG_SKIP_FIRST_LOAD) ? star::kDebugSkipFirstLoad : 0;
   cudaError_t e = star::set_debug_attn(limit, dev_flags);
   if (e == cudaSuccess) e = star::set_debug_decode(limit, dev_flags);
+  if (e == cudaSuccess) e = star::set_debug_exchange(limit, 0);
   return e == cudaSuccess ? STAR_OK : cuda_fail(e, "debug settings");
 }
 

@@ -20,7 +20,7 @@
 //
 // CTA organisation (384 threads, persistent, one CTA per SM):
 //   warp 0      TMA producer: K and V tiles from the paged cache into two
-//               shared-memory rings (128-byte swizzle, no multicast).
+//               shared-memory rings (128-byte swizzle; each CTA loads its own tiles).
 //   warp 1      MMA issuer: S_w = Q_w K^T (SS form) and O_w += P_w V (A from TMEM).
 //   warps 4-7   softmax warpgroup 0 (Q tile 0: rows <-> TMEM lanes 0..127)
 //   warps 8-11  softmax warpgroup 1 (Q tile 1)

@@ -39,6 +39,7 @@ enum DeviceError : int {
   kDevTimeoutSoftmax = 3,
   kDevBadPage = 4,
   kDevBadPartial = 5,   // a merged partial had a NaN or +inf LSE (skipped, like an empty one)
+  kDevTimeoutExchange = 6,  // a peer-exchange wait (another rank's ready or ack word) ran out
 };
 static __device__ int g_device_error = 0;
 
@@ -140,7 +141,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int er
 }
 
 // ---------------------------------------------------------------------------
-// TMA (tiled tensor loads, no multicast)
+// TMA (tiled tensor loads into this CTA's own shared memory)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tma_load_4d(void* smem_dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
                                             int c2, int c3) {

@@ -32,7 +32,7 @@
 // mbarrier that the producer waits on before the tile holding that slot.
 //
 // CTA (256 threads, one per SM):
-//   warp 0     TMA producer (K and V rings, no multicast)
+//   warp 0     TMA producer (K and V rings, loaded by this CTA only)
 //   warp 1     TMEM allocation and MMA issuer
 //   warps 2-7  prologue (append, q) while warp 0 already streams K and V
 //   warps 4-7  then softmax and O accumulation: thread = TMEM lane 32 (w - 4) + lane

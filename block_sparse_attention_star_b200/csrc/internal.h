@@ -146,6 +146,21 @@ int decode_pick_chunk(int B, int Hkv, int G, int n_keys, int num_sms);
 int decode_pick_chunk_var(int B, int Hkv, const int* n_keys_of, int min_chunk, int num_sms);
 cudaError_t launch_decode(const DecodeLaunch& a, cudaStream_t st);
 
+// --- exchange.cu: the Phase-2 star exchange over peer memory ---------------------
+struct ExchangeView {
+  int world, rank, slots;   // ranks, this rank, partials per rank per exchange
+  void* peers[8];           // every rank's exchange buffer as mapped in this process
+};
+size_t exchange_bytes(int world, int slots, long long rows, int d);
+// Merge n_groups groups of ppg chunk partials (o_in [n_groups*ppg][rows][d], lse_in) into
+// slots [0, n_groups) (empty partials in [n_groups, slots)) and store them into slot `rank`
+// of every rank's buffer, parity epoch & 1; then publish ready = epoch.
+cudaError_t launch_merge_scatter(const ExchangeView& x, int n_groups, int ppg, long long rows, int d,
+                                 const float* o_in, const float* lse_in, unsigned long long epoch, cudaStream_t st);
+// Wait for every rank's slot of the epoch in this rank's buffer, merge, ack.
+cudaError_t launch_gather_merge(const ExchangeView& x, long long rows, int d, unsigned long long epoch, void* out,
+                                float* lse_out, cudaStream_t st);
+
 // --- api.cu: the thread-local message read by star_last_error(); returns code ----
 int set_last_error(int code, const char* msg);
 
@@ -154,9 +169,11 @@ cudaError_t read_and_clear_error_attn(int* code);
 cudaError_t read_and_clear_error_decode(int* code);
 cudaError_t read_and_clear_error_rope(int* code);
 cudaError_t read_and_clear_error_merge(int* code);
+cudaError_t read_and_clear_error_exchange(int* code);
 
 // --- failure-detection test hooks (per kernel file; see common.cuh) -------------
 cudaError_t set_debug_attn(unsigned long long wait_limit_ns, int flags);
 cudaError_t set_debug_decode(unsigned long long wait_limit_ns, int flags);
+cudaError_t set_debug_exchange(unsigned long long wait_limit_ns, int flags);
 
 }  // namespace star

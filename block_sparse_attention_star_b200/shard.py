@@ -20,6 +20,7 @@ start, and the merge waits only for its own gathers (no barrier).
 
 from __future__ import annotations
 
+import ctypes
 import math
 from typing import Callable
 
@@ -128,3 +129,56 @@ class ShardExchange:
             lse_out = torch.empty((rows,), dtype=torch.float32, device=o_all.device)
         star_lse_merge(P, rows, d, o_all, lse_all, out.view(rows, d), lse_out.view(rows))
         return out, lse_out
+
+
+class PeerExchange:
+    """One rank's exchange over peer memory (star.h star_exchange): the kernels that finish a
+    shard's partials store them straight into every rank's buffer over NVLink, and
+    ``star_exchange_merge`` waits for them in this rank's own buffer and merges (no collective
+    library on the data path; torch.distributed only carries the buffers' IPC handles once).
+
+    rows, d, slots: the shape of one exchange (rows x d per partial, slots partials per rank).
+    Epochs count this exchange's uses, 1, 2, ..., the same on every rank.
+    """
+
+    def __init__(self, rows: int, d: int, slots: int, group=None, device="cuda"):
+        from . import StarExchange, star_exchange_size, star_ipc_export, star_ipc_open
+        self.dist = dist.is_available() and dist.is_initialized()
+        self.world = dist.get_world_size(group) if self.dist else 1
+        self.rank = dist.get_rank(group) if self.dist else 0
+        if self.world > 8:
+            raise ValueError("the peer exchange serves up to 8 ranks (one NVLink domain of one node)")
+        self.rows, self.d, self.slots = rows, d, slots
+        size = star_exchange_size(self.world, slots, rows, d)
+        self.buf = torch.zeros(size + 256, dtype=torch.uint8, device=device)
+        base = self.buf.data_ptr()
+        self.local = self.buf[(-base) % 256:]  # 256-byte aligned start
+        ptrs = [0] * self.world
+        ptrs[self.rank] = self.local.data_ptr()
+        self.opened: list[tuple[int, int]] = []
+        if self.world > 1:
+            torch.cuda.synchronize(device)  # the zero fill is done before any peer writes
+            mine = star_ipc_export(self.local)
+            handles = [None] * self.world
+            dist.all_gather_object(handles, mine, group=group)
+            for w, (h, off) in enumerate(handles):
+                if w != self.rank:
+                    ptrs[w] = star_ipc_open(h, off)
+                    self.opened.append((ptrs[w], off))
+            dist.barrier(group=group)  # every buffer is zeroed and mapped before the first push
+        self.ex = StarExchange(self.world, self.rank, slots, (ctypes.c_void_p * 8)(*ptrs))
+        self.epoch = 0
+
+    def next_epoch(self) -> int:
+        self.epoch += 1
+        return self.epoch
+
+    def merge(self, out, lse_out=None, epoch: int | None = None):
+        from . import star_exchange_merge
+        star_exchange_merge(self.ex, self.rows, self.d, self.epoch if epoch is None else epoch, out, lse_out)
+
+    def close(self):
+        from . import star_ipc_close
+        for ptr, off in self.opened:
+            star_ipc_close(ptr, off)
+        self.opened = []

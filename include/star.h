@@ -56,7 +56,7 @@ enum {
 };
 
 /* Workspace query selectors. */
-enum { STAR_OP_PHASE1 = 1, STAR_OP_PHASE2 = 2, STAR_OP_DECODE = 3, STAR_OP_PHASE1_ANCHOR = 4 };
+enum { STAR_OP_PHASE1 = 1, STAR_OP_PHASE2 = 2, STAR_OP_DECODE = 3, STAR_OP_PHASE1_ANCHOR = 4, STAR_OP_PHASE2_PUSH = 5 };
 
 /* Problem shape ("问题定义与记号": context c of n blocks of b tokens, query q). */
 typedef struct star_shape {
@@ -121,8 +121,9 @@ int star_page_table_fill(const star_shape* shape, int32_t* page_table_host, int3
  * STAR_OP_PHASE1: 0.  STAR_OP_PHASE1_ANCHOR: star_phase1_encode_anchored with anchor
  * position ids, B*(n-1)*Hkv*a*d*2 bytes (the anchor's keys roped at those ids).
  * STAR_OP_PHASE2: RoPE(q) (B*T*Hq*d*2 bytes, rounded up to 256), plus the f32 partials
- * of the chunks when blocks are split to fill the GPU.  STAR_OP_DECODE: the chunk
- * partials of one step. */
+ * of the chunks when blocks are split to fill the GPU.  STAR_OP_PHASE2_PUSH: the same
+ * with the chunk partials always staged (star_phase2_partial_shard_push).
+ * STAR_OP_DECODE: the chunk partials of one step. */
 int star_workspace_size(const star_shape* shape, int op, int32_t T, size_t* bytes_out);
 
 /* Integer structure of c' ("被增广的上下文"), for checking only.
@@ -309,6 +310,61 @@ int star_phase2_partial_shard(const star_shape* shape, const star_cache* cache, 
 int star_decode_partial_shard(const star_shape* shape, const star_cache* cache, const star_shard* shard, const void* q,
                               const void* k, const void* v, const int32_t* pos, int32_t cur_len, float* o_part,
                               float* lse_part, void* ws, size_t ws_bytes, star_stream_t stream);
+
+/* The exchange over peer memory (NVLink): instead of gathering the partials with a
+ * collective library, the kernel that finishes a shard's partials stores them straight
+ * into every GPU's exchange buffer, and the merge waits for them there.
+ *
+ * Each rank allocates ONE exchange buffer of star_exchange_size(world, slots, rows, d)
+ * bytes in its own device memory, zero-filled once before its first use (afterwards the
+ * calls keep it consistent), maps every other rank's buffer into its process
+ * (star_ipc_export / star_ipc_open; peers[w] = rank w's buffer, peers[rank] = its own),
+ * and numbers its exchanges 1, 2, 3, ... (epoch), in the same order on every rank.
+ * Exchange e uses parity e & 1 of every buffer; a push of epoch e first waits until every
+ * rank has merged epoch e - 2 (no barrier).  Every wait is bounded (2 s): a rank that
+ * never arrives makes the waiting kernel record STAR_ERR_TIMEOUT (star_device_status) and
+ * return.  One buffer serves one kind of exchange (one rows x slots shape). */
+typedef struct star_exchange {
+  int32_t world;    /* ranks, 1..8 */
+  int32_t rank;     /* this rank */
+  int32_t slots;    /* partials each rank contributes per exchange (ceil(n / world) for Phase 2, 1 for decode) */
+  void* peers[8];   /* device addresses of every rank's exchange buffer as mapped here; 256-byte aligned */
+} star_exchange;
+
+/* Bytes of one rank's exchange buffer for exchanges of `slots` partials of `rows` rows of
+ * head dim d per rank: a 256-byte header plus 2 x world x (slots*rows*(d+1)*4, each part
+ * rounded up to 256). */
+int star_exchange_size(int32_t world, int32_t slots, int64_t rows, int32_t d, size_t* bytes_out);
+
+/* star_phase2_partial_shard, with the shard's per-block partials pushed into slot `rank` of
+ * every rank's exchange buffer (epoch) instead of written to o_part / lse_part; the slots
+ * past the shard's blocks get empty partials (O = 0, LSE = -inf).  rows = B*T*Hq.
+ * ws: star_workspace_size(STAR_OP_PHASE2_PUSH, T) bytes.  ex->slots >= the shard's blocks. */
+int star_phase2_partial_shard_push(const star_shape* shape, const star_cache* cache, const star_shard* shard,
+                                   const void* q, const void* k, const void* v, const int32_t* q_pos, int32_t T,
+                                   const star_exchange* ex, uint64_t epoch, void* ws, size_t ws_bytes,
+                                   star_stream_t stream);
+
+/* star_decode_partial_shard, with the shard's (O, LSE) pushed into slot `rank` of every
+ * rank's exchange buffer (one slot, rows = B*Hq).  ws: star_workspace_size(STAR_OP_DECODE). */
+int star_decode_partial_shard_push(const star_shape* shape, const star_cache* cache, const star_shard* shard,
+                                   const void* q, const void* k, const void* v, const int32_t* pos, int32_t cur_len,
+                                   const star_exchange* ex, uint64_t epoch, void* ws, size_t ws_bytes,
+                                   star_stream_t stream);
+
+/* Waits until every rank's partials of `epoch` are in this rank's buffer, merges the
+ * world x slots partials of each row ("组装全局结果", log-sum-exp form of "数值稳定性") into
+ * out (bf16 [rows][d]) and lse_out (f32 [rows], may be NULL), then tells every rank that
+ * this rank's slots of the epoch's parity may be reused. */
+int star_exchange_merge(const star_exchange* ex, int64_t rows, int32_t d, uint64_t epoch, void* out, float* lse_out,
+                        star_stream_t stream);
+
+/* CUDA IPC for the exchange buffers (host calls): export a device pointer of this process
+ * as a 64-byte handle plus its offset in its allocation; open a peer's handle (the pointer
+ * is valid in this process, peer access enabled); close it when done. */
+int star_ipc_export(const void* ptr, void* handle_out /* 64 bytes */, uint64_t* offset_out);
+int star_ipc_open(const void* handle /* 64 bytes */, uint64_t offset, void** ptr_out);
+int star_ipc_close(void* ptr, uint64_t offset);
 
 /* Tracing: when both are non-NULL (cudaEvent_t handles created by the caller),
  * every later call on this thread records `start_event` on its stream right

@@ -151,3 +151,19 @@ def test_encode_layers_callback_marshalling_without_a_launch():
         star._check(star.lib().star_encode_layers(ctypes.byref(sh), 1, ctypes.byref(FakeCache.c), None, None, None,
                                                   None, None, None, star.LAYER_FN(), None, None))
     assert e.value.code == star.STAR_ERR_INVALID_ARG
+
+
+def test_exchange_buffer_size_and_checks():
+    """The peer-exchange buffer: a 256-byte header, then 2 parities x world slots of
+    slots x rows partials (f32 O rows of d, then f32 LSEs), each part rounded up to 256 bytes."""
+    import block_sparse_attention_star_b200 as star
+    def rup(x):
+        return (x + 255) // 256 * 256
+    for world, slots, rows, d in [(1, 4, 2048, 128), (2, 2, 2048, 128), (8, 1, 32, 128), (3, 5, 7, 64)]:
+        slot = rup(slots * rows * d * 4) + rup(slots * rows * 4)
+        assert star.star_exchange_size(world, slots, rows, d) == 256 + 2 * world * slot
+    for bad, code in [((9, 1, 32, 128), star.STAR_ERR_UNSUPPORTED_SHAPE), ((2, 0, 32, 128), star.STAR_ERR_INVALID_ARG),
+                      ((2, 1, 32, 96), star.STAR_ERR_UNSUPPORTED_SHAPE)]:
+        with pytest.raises(star.StarError) as e:
+            star.star_exchange_size(*bad)
+        assert e.value.code == code
