@@ -38,8 +38,10 @@ def _buffers(star, world, slots, rows, d):
     return bufs, views
 
 
-@pytest.mark.parametrize("world", [1, 2])
+@pytest.mark.parametrize("world", [1, 2, 3])
 def test_peer_exchange_matches_the_oracle(world):
+    """world 3 splits the 4 blocks 2 + 1 + 1: the ranks with one block pad their second slot
+    with an empty partial."""
     import block_sparse_attention_star_b200 as star
     from block_sparse_attention_star_b200.shard import block_range
     from tests import harness as h
