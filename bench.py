@@ -40,6 +40,9 @@ sys.path.insert(0, ROOT)
 from synth import get_config, make_inputs  # noqa: E402
 
 METRIC = "Phase-1 ctx tok/s (% BF16 peak) at 128K; Phase-2 decode µs/step (HBM GB/s)"
+# Datasheet figures for one B200, for the nominal fractions beside the measured ones: dense bf16
+# tensor throughput (NVIDIA's 2:4-sparse figure halved) and HBM3e bandwidth (about 8 TB/s).
+NOMINAL = {"bf16_tflops": 2250.0, "hbm_gbs": 8000.0}
 UNIT = "ctx tok/s"
 
 
@@ -537,12 +540,14 @@ def run_star(args, rank, world, local_rank):
         "data": "synthetic (seeded N(0,1) bf16; 1% of context key rows x8 where the workload says peaky)",
         "config": workload_config(wl, world),
         "phase1": {"attn_ms": p1_ms, "ctx_tok_s": wl.context_tokens() / (p1_ms * 1e-3), "tflops": tflops,
-                   "frac_bf16_burst": tflops / peaks["bf16"], "frac_bf16_sustained": tflops / peaks["bf16_sustained"]},
+                   "frac_bf16_burst": tflops / peaks["bf16"], "frac_bf16_sustained": tflops / peaks["bf16_sustained"],
+                   "frac_bf16_nominal": tflops / NOMINAL["bf16_tflops"]},
         "phase2": phase2_roofline(wl, run.shape.n, p2_ms, peaks),
         "query_merge": merge_roofline(wl.B * wl.T * wl.Hq, run.shape.n, wl.d, merge_ms, peaks),
         "decode": {"us_per_step": 1e3 * dec_step_ms, "kernel_us": 1e3 * statistics.mean(dec_kernel_ms),
                    "bytes_per_step": dec_bytes, "kernel_gbs": dec_gbs, "frac_hbm": dec_gbs / peaks["hbm_gbs"],
                    "step_gbs": dec_bytes / (dec_step_ms * 1e-3) / 1e9,
+                   "frac_hbm_nominal": dec_gbs / NOMINAL["hbm_gbs"],
                    "timing": "us_per_step: the S steps' span in the timed region / S (append, attention, merge "
                              "and launch gaps); kernel_us: the attention kernel alone, one extra untimed step"},
         "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16"], "unit": "TFLOP/s",
