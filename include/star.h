@@ -23,7 +23,9 @@
  *     `ws` of at least star_workspace_size() bytes.
  *   - Every call is asynchronous on the caller's CUDA stream `stream` (a
  *     cudaStream_t; NULL = legacy default stream) and never synchronises, except
- *     star_device_status().
+ *     star_device_status().  The compute calls can be captured into a CUDA graph
+ *     once each has run eagerly on the device (the first call of a kernel sets its
+ *     shared-memory opt-in); a replay recomputes from the buffers' current contents.
  *   - Return value: STAR_OK (0) or a negative STAR_ERR_* code; star_last_error()
  *     then describes the failure (thread-local).  Arguments are validated on the
  *     host before anything is launched; a failing call launches nothing.
