@@ -167,3 +167,14 @@ def test_exchange_buffer_size_and_checks():
         with pytest.raises(star.StarError) as e:
             star.star_exchange_size(*bad)
         assert e.value.code == code
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """No fallback: without libstar.so every call raises instead of computing anything."""
+    monkeypatch.setattr(star, "_lib", None)
+    monkeypatch.setattr(star, "LIB_PATH", str(tmp_path / "libstar.so"))
+    with pytest.raises(ImportError, match="missing"):
+        star.star_version()
+    with pytest.raises(ImportError, match="missing"):
+        star.star_lse_merge(1, 1, 128, torch.zeros(1, 1, 128), torch.zeros(1, 1), torch.zeros(1, 128),
+                            torch.zeros(1))
