@@ -5,7 +5,8 @@ the decode steps with their appends) is a sequence of kernel launches on the cal
 stream with no allocation and no host synchronisation, so it can be captured once a
 first call has set up each kernel (shared-memory opt-ins).  A replay recomputes the
 step from the same inputs: every output must be bit-identical to the eager run, and
-two replays to each other.
+two replays to each other (context anchors at caller ids and per-sequence lengths
+included).
 """
 
 import dataclasses
@@ -31,15 +32,20 @@ def _outputs(run):
 
 
 def _poison(run):
+    # the same sentinel before the eager step and before each replay, so that rows no
+    # step writes (past a shorter sequence's context) compare equal
     for n in OUTS:
-        t = getattr(run, n)
-        t.fill_(float("nan"))
+        getattr(run, n).fill_(-7.0)
 
 
 @pytest.mark.parametrize("wl", [
     get_config("tiny"),
     Workload("d128-g4-b2-graph", B=2, Hq=8, Hkv=2, d=128, L=2048, b=512, T=40, S=5, peaky=True),
     dataclasses.replace(get_config("llama8b-32k"), S=4),
+    Workload("graph-anchor-offset", B=1, Hq=8, Hkv=2, d=128, L=2048, b=512, T=16, S=3, peaky=False,
+             anchor=256, anchor_ids="offset"),
+    Workload("graph-varlen", B=3, Hq=8, Hkv=2, d=128, L=2048, b=512, T=16, S=3, peaky=True,
+             seq_lens=(2048, 1500, 700)),
 ], ids=lambda w: w.name)
 def test_step_replays_bit_identically(wl):
     import block_sparse_attention_star_b200 as star
@@ -47,6 +53,7 @@ def test_step_replays_bit_identically(wl):
 
     dev = torch.device("cuda", 0)
     run = StarRun(wl, dev)
+    _poison(run)
     run.step()  # eager: sets up every kernel before capture
     torch.cuda.synchronize()
     assert star.star_device_status() == 0

@@ -38,6 +38,10 @@ SMALL = {
     "d128-g8-t130": Workload("d128-g8-t130", B=1, Hq=16, Hkv=2, d=128, L=1024, b=256, T=130, S=2, peaky=True),
     "d64-g2-p128": Workload("d64-g2-p128", B=1, Hq=4, Hkv=2, d=64, L=768, b=256, T=7, S=4, peaky=False,
                             page_tokens=128),
+    # one query token; the decode slots and the query tail cross page boundaries (pages of 256)
+    "d128-t1": Workload("d128-t1", B=1, Hq=8, Hkv=2, d=128, L=1024, b=256, T=1, S=3, peaky=True),
+    "d128-pagecross": Workload("d128-pagecross", B=2, Hq=8, Hkv=2, d=128, L=1024, b=256, T=250, S=10,
+                               peaky=False),
 }
 
 
