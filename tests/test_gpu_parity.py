@@ -42,6 +42,9 @@ SMALL = {
     "d128-t1": Workload("d128-t1", B=1, Hq=8, Hkv=2, d=128, L=1024, b=256, T=1, S=3, peaky=True),
     "d128-pagecross": Workload("d128-pagecross", B=2, Hq=8, Hkv=2, d=128, L=1024, b=256, T=250, S=10,
                                peaky=False),
+    "d64-g8": Workload("d64-g8", B=1, Hq=16, Hkv=2, d=64, L=1024, b=256, T=24, S=3, peaky=True),
+    "d128-p512": Workload("d128-p512", B=1, Hq=8, Hkv=2, d=128, L=2048, b=512, T=16, S=3, peaky=False,
+                          page_tokens=512),
 }
 
 
