@@ -36,6 +36,8 @@ def _shape(**kw):
     (dict(anchor=-128), star.STAR_ERR_INVALID_ARG),              # negative anchor size
     (dict(anchor=1000), star.STAR_ERR_UNSUPPORTED_SHAPE),         # anchor not a multiple of 128
     (dict(anchor=32768 + 128), star.STAR_ERR_UNSUPPORTED_SHAPE),  # anchor larger than the block
+    (dict(B=2, seq_len=(0, 131072)), star.STAR_ERR_INVALID_ARG),   # an empty context
+    (dict(seq_len=(131072 + 1,)), star.STAR_ERR_INVALID_ARG),      # longer than the capacity L
 ])
 def test_shape_validation(kw, code):
     with pytest.raises(star.StarError) as e:
